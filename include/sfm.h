@@ -1,0 +1,209 @@
+/*
+ * sfm.h -- C ABI of the performer's next-unit flow-matching denoising step
+ * (Wan-Streamer v0.2) on one NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute.  The pages describe the performer's per-unit work
+ * without signatures: the thinker broadcasts a compact, performer-compatible
+ * K/V slice; each performer rank writes it into a pre-allocated local cache;
+ * the performer then runs the flow-matching solver over the next unit's audio
+ * and video latents and returns them ("Wan-Streamer v0.2: Higher Resolution,
+ * Same Latency" digest, "method overview and architecture"; "Wan-Streamer
+ * v0.2" blog, "Infra"; v0.2 abstract).  The solver integrates the
+ * rectified-flow path z_tau = (1 - tau) z0 + tau eps from tau = 1 to tau = 0
+ * with Euler steps z <- z + (tau_next - tau) v, v = f_theta(z, tau | cache)
+ * ("Wan-Streamer" v0.1 blog, §3.4 conditional flow matching), where f_theta is
+ * the block-causal Transformer of §3.3: the current unit's tokens see every
+ * cached unit and each other (bidirectional inside the unit).
+ *
+ * Conventions for every call:
+ *   - Plain pointers.  "device" = CUDA device memory of the current device,
+ *     "host" = ordinary host memory.  Matrices are row-major; a weight matrix
+ *     W of a linear map x -> x W^T is stored [out][in].
+ *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on that stream: device buffers passed in must
+ *     stay valid and unmodified until the stream has executed the call.
+ *   - Every argument, session and capacity error is detected on the host
+ *     BEFORE any launch and returned as a negative status; nothing is
+ *     written in that case.  A CUDA launch failure returns SFM_ECUDA;
+ *     asynchronous device errors surface on a later call.  No call aborts the
+ *     process or throws across the ABI.
+ *   - One handle is used by one host thread / one stream at a time.
+ */
+#ifndef SFM_H_
+#define SFM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define SFM_OK             0
+#define SFM_EINVAL        (-1)   /* bad argument (null pointer, size, shape)      */
+#define SFM_ECAPACITY     (-2)   /* cache or pool full (ring off), batch too big  */
+#define SFM_ESESSION      (-3)   /* session id not open                           */
+#define SFM_ECUDA         (-4)   /* a CUDA call failed (see sfm_last_cuda_error)  */
+#define SFM_ENOMEM        (-5)   /* device allocation failed in sfm_create        */
+#define SFM_EUNSUPPORTED  (-6)   /* shape the kernels do not support              */
+
+/* ---- storage / arithmetic type of weights, cache and activations -------- */
+#define SFM_DTYPE_BF16 0   /* bf16 storage, tensor-core MMA with fp32 accumulation;
+                              residual stream, softmax, z and v in fp32           */
+#define SFM_DTYPE_FP32 1   /* fp32 everywhere (CUDA cores); small shapes          */
+
+typedef struct sfm_handle sfm_handle;   /* opaque, library-owned */
+
+/* Shapes of f_theta and of one streaming unit. */
+typedef struct sfm_config {
+  int n_layers;          /* L                                                   */
+  int d_model;           /* d: multiple of 64                                   */
+  int n_heads;           /* H                                                   */
+  int head_dim;          /* D_h: 128 for bf16; even and <= 128 for fp32         */
+  int d_mlp;             /* F: multiple of 64                                   */
+  int c_lat;             /* C: latent channels per token (<= 64)                */
+  int n_video;           /* video tokens of the current unit (raster order)     */
+  int n_audio;           /* audio tokens of the current unit (after the video)  */
+  int unit_kv_tokens;    /* T_u: K/V tokens the thinker sends per unit          */
+  int max_sessions;      /* sessions open at once; also the largest batch       */
+  long long pool_tokens; /* per-layer K/V rows of the cache pool shared by all
+                            sessions; a session with capacity U units takes
+                            U * T_u + (n_video + n_audio) rows                  */
+  int dtype;             /* SFM_DTYPE_BF16 | SFM_DTYPE_FP32                     */
+  int ring;              /* 1: a full session cache overwrites its oldest unit;
+                            0: sfm_kvcache_append returns SFM_ECAPACITY          */
+  double rope_theta;     /* RoPE base (10000)                                   */
+  double rms_eps;        /* RMSNorm epsilon (1e-6)                              */
+} sfm_config;
+
+/*
+ * Weights of f_theta: device pointers of the config's dtype, borrowed (not
+ * copied) for the handle's lifetime.  The per-layer members are HOST arrays
+ * of n_layers device pointers; the arrays themselves are copied at create.
+ *   w_in   [d][C]           x_j = W_in z_j + e_mod[m(j)] + temb(tau)
+ *   e_mod  [2][d]           row 0 video, row 1 audio
+ *   g_final[d], w_out[C][d] v = RMSNorm(x; g_final) W_out^T
+ *   g_attn [d]              pre-attention RMSNorm gain
+ *   w_qkv  [3 H D_h][d]     output rows: q (head-major, D_h per head), then k, then v
+ *   w_o    [d][H D_h]
+ *   g_mlp  [d]              pre-MLP RMSNorm gain
+ *   w_1    [F][d], w_2 [d][F]   x += GELU_tanh(RMSNorm(x) W_1^T) W_2^T
+ * A handle created with w == NULL supports only the cache calls.
+ */
+typedef struct sfm_weights {
+  const void* w_in;
+  const void* e_mod;
+  const void* g_final;
+  const void* w_out;
+  const void* const* g_attn;
+  const void* const* w_qkv;
+  const void* const* w_o;
+  const void* const* g_mlp;
+  const void* const* w_1;
+  const void* const* w_2;
+} sfm_weights;
+
+/* Per-session cache bookkeeping (host copy). */
+typedef struct sfm_session_info {
+  int cache_units;          /* capacity in units (slots)                          */
+  long long units_appended; /* units ever appended, evicted ones included         */
+  long long valid_tokens;   /* min(units_appended, cache_units) * T_u             */
+  long long p0;             /* position of the current unit's first token
+                               = units_appended * T_u                             */
+  long long base_row;       /* first pool row of this session                     */
+} sfm_session_info;
+
+/* ---- handle ------------------------------------------------------------- */
+
+/* Validates cfg, allocates the K/V pool (2 * L * pool_tokens * H * D_h
+ * elements) and all scratch on the current device.  Returns SFM_EINVAL /
+ * SFM_EUNSUPPORTED for bad shapes, SFM_ENOMEM if allocation fails.  The hot
+ * path allocates nothing after this call. */
+int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out);
+
+/* Frees everything the handle owns (synchronises the device first). */
+void sfm_destroy(sfm_handle* h);
+
+/* Carves a contiguous cache region of cache_units unit slots (plus the
+ * current unit's scratch rows) out of the pool for a new session.
+ * SFM_ECAPACITY if the pool or the session table is full. */
+int sfm_session_open(sfm_handle* h, int cache_units, int* session);
+
+/* Forgets a session's units (counters to zero); its region stays reserved. */
+int sfm_session_reset(sfm_handle* h, int session);
+
+int sfm_session_get_info(const sfm_handle* h, int session, sfm_session_info* out);
+
+/* ---- the hot path ------------------------------------------------------- */
+
+/*
+ * Writes the thinker's K/V slice for n_tok / T_u whole units into the
+ * session's cache: unit u (u = units_appended + i) goes to slot u mod
+ * cache_units, rows verbatim.  k, v: device, [L][n_tok][H][D_h] of the
+ * handle's dtype, caller-owned; K is already rotated (post-RoPE).
+ * SFM_EINVAL if n_tok is not a positive multiple of T_u; SFM_ECAPACITY if
+ * ring == 0 and the units do not fit (nothing is written).
+ */
+int sfm_kvcache_append(sfm_handle* h, int session, const void* k, const void* v,
+                       int n_tok, void* stream);
+
+/* Copies cache rows [row0, row0 + n_rows) of one layer into caller device
+ * buffers k_dst, v_dst ([n_rows][H][D_h]).  Rows index the session's region
+ * (slot s occupies rows [s T_u, (s+1) T_u)). */
+int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long long row0,
+                     long long n_rows, void* k_dst, void* v_dst, void* stream);
+
+/*
+ * One Euler step of the current unit: v = f_theta(z, tau_from | cache),
+ * z <- z + (tau_to - tau_from) v.  z: device fp32 [N][C], N = n_video +
+ * n_audio (video rows first), updated in place.  v_out: nullable device fp32
+ * [N][C] receiving v.  The current unit's tokens are at positions p0 + j.
+ */
+int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_from,
+                     float tau_to, float* v_out, void* stream);
+
+/*
+ * The whole solve: Euler steps over taus[0] -> taus[1] -> ... -> taus[n-1].
+ * taus: host array, n_taus >= 2, taus[0] = 1 (z holds eps) decreasing to
+ * taus[n-1] = 0 (z then holds the unit's clean latent).  The cache is not
+ * modified (the current unit's K/V are scratch, never committed).
+ */
+int sfm_fm_solve(sfm_handle* h, int session, float* z, const float* taus,
+                 int n_taus, void* stream);
+
+/* Batched solve over n_sessions open sessions (distinct ids), each with its
+ * own cache length; z[i] is session i's device fp32 [N][C].  sessions and z
+ * are host arrays.  SFM_ECAPACITY if n_sessions > max_sessions. */
+int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions,
+                         float* const* z, const float* taus, int n_taus, void* stream);
+
+/* ---- standalone kernels --------------------------------------------------- */
+
+/*
+ * Softmax attention O = softmax(Q K^T / sqrt(D_h)) V per head, every key
+ * visible to every query (the performer form of block-causal attention: all
+ * keys are cached units <= the current one or the current unit itself).
+ * q: [n_q][H][D_h], k, v: [n_kv][H][D_h], o: [n_q][H][D_h], device, dtype as
+ * given.  workspace: device scratch of at least
+ * sfm_attention_workspace_bytes(...) bytes (caller-owned; may be NULL when
+ * that size is 0).  n_kv >= 1.
+ */
+size_t sfm_attention_workspace_bytes(int n_q, int n_kv, int n_heads, int head_dim, int dtype);
+int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q, int n_kv,
+                  int n_heads, int head_dim, int dtype, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/* Vectorised Euler update z[i] += dtau * v[i], i < n; device fp32. */
+int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream);
+
+/* ---- errors --------------------------------------------------------------- */
+const char* sfm_strerror(int status);
+/* The cudaError_t of the last failed CUDA call made by this library on this
+ * host thread (0 if none). */
+int sfm_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SFM_H_ */

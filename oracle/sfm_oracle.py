@@ -1,0 +1,369 @@
+"""fp64 CPU oracle for the performer's next-unit flow-matching denoising step.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import or run
+this module.  The product path (``streaming_flow_matching_b200``) never calls
+it, and this module imports nothing from the product: the two share no code.
+
+Plain, slow, obviously correct: numpy float64 throughout, one function per step
+of the method, written in the order the pages give it.  A library matmul is the
+only primitive used; there is no blocking, fusion or reordering.  bf16 inputs are
+upcast exactly to float64; no intermediate bf16 rounding is emulated.
+
+Sources (the pages are web write-ups of Wan-Streamer; none prints code):
+  [v0.1]  "Wan-Streamer" blog (gongshangzheng.github.io): §3.1 streaming
+          formulation, §3.3 block-causal Transformer, §3.4 conditional flow
+          matching, Fig. 2 thinker/performer timeline.
+  [dig]   "Wan-Streamer v0.2: Higher Resolution, Same Latency" digest
+          (nanless.github.io): "method overview and architecture" (performer
+          path, pre-sharded K/V cache, audio unsharded), "details" (step count,
+          noise schedule undisclosed).
+  [blog]  "Wan-Streamer v0.2" blog (zhao9797.github.io): "Infra" section.
+  [abs]   "Wan-Streamer v0.2" abstract (chatpaper.ai).
+
+Readings taken where the pages are silent (each also listed in the design doc):
+  * rectified-flow path z_tau = (1 - tau) z0 + tau eps, velocity eps - z0
+    (the path formula of [v0.1] §3.4 was lost in extraction; the symbol glosses
+    survive); Euler solve from tau = 1 to tau = 0, z <- z + (tau_next - tau) v.
+  * uniform step schedule (the count is undisclosed, [dig] "details").
+  * tau enters f_theta through a parameter-free sinusoidal embedding added to
+    every token at the input.
+  * pre-norm blocks: RMSNorm -> QKV -> 1-D rotate-half RoPE -> softmax
+    attention -> O-proj + residual; RMSNorm -> W1 -> tanh-GELU -> W2 + residual;
+    final RMSNorm -> velocity head.  No biases.
+  * cached K is stored post-RoPE (the thinker builds it), so it is never rotated
+    here; current-unit tokens sit at absolute positions P0 + j, P0 = tokens ever
+    appended to the session.
+  * token order inside the current unit: video raster first, then audio.
+  * ring cache: unit u lands in slot u mod n_slots.
+
+Parity status: every step is pinned by tests in ``tests/test_oracle_pins.py``
+(closed forms, invariants, brute force at tiny sizes, library routines).  The
+composed velocity network f_theta has no published values to pin against; it is
+pinned by a scalar-loop brute-force re-derivation at tiny size, by the
+block-causal consistency check (performer form == masked full-sequence form),
+and by invariants.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+VIDEO, AUDIO = 0, 1
+
+
+def f64(a):
+    """Upcast an array-like (numpy, or a CPU torch tensor of any dtype) to float64."""
+    if hasattr(a, "detach"):
+        return a.detach().to("cpu").double().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+@dataclass
+class Config:
+    """Shapes of f_theta and of one streaming unit."""
+    n_layers: int
+    d_model: int
+    n_heads: int
+    head_dim: int
+    d_mlp: int
+    c_lat: int
+    n_video: int
+    n_audio: int
+    unit_kv_tokens: int
+    rope_theta: float = 10000.0
+    rms_eps: float = 1e-6
+
+    @property
+    def n_tokens(self) -> int:
+        return self.n_video + self.n_audio
+
+    @property
+    def hd(self) -> int:
+        return self.n_heads * self.head_dim
+
+
+# ---------------------------------------------------------------------------
+# elementwise pieces
+# ---------------------------------------------------------------------------
+
+def rmsnorm(x, g, eps):
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * g (pre-norm block)."""
+    x = f64(x)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * f64(g)
+
+
+def gelu_tanh(x):
+    """tanh approximation of GELU: 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))."""
+    x = f64(x)
+    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def rope_freqs(head_dim, theta):
+    """omega_i = theta^(-2 i / head_dim) for i < head_dim / 2."""
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return theta ** (-2.0 * i / head_dim)
+
+
+def rope(x, pos, theta):
+    """1-D rotary embedding, rotate-half pairing (i, i + D/2).
+
+    x: [N][H][D]; pos: [N] absolute positions.  Pair (a, b) = (x_i, x_{i+D/2})
+    rotated by angle pos * omega_i:  a' = a cos - b sin,  b' = b cos + a sin.
+    """
+    x = f64(x)
+    d = x.shape[-1]
+    half = d // 2
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * rope_freqs(d, theta)[None, :]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    a = x[..., :half]
+    b = x[..., half:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def tau_embedding(tau, d):
+    """Parameter-free sinusoidal embedding of the flow time tau.
+
+    e_i = sin(1000 tau w_i) for i < d/2 and e_i = cos(1000 tau w_{i-d/2}) for
+    i >= d/2, with w_i = 10000^(-2 i / d).
+    """
+    half = d // 2
+    w = 10000.0 ** (-2.0 * np.arange(half, dtype=np.float64) / d)
+    ang = 1000.0 * float(tau) * w
+    return np.concatenate([np.sin(ang), np.cos(ang)])
+
+
+def modality_of_tokens(cfg: Config):
+    """Modality id per current-unit token: video raster tokens, then audio tokens."""
+    m = np.full(cfg.n_tokens, VIDEO, dtype=np.int64)
+    m[cfg.n_video:] = AUDIO
+    return m
+
+
+def linear(x, w):
+    """y = x W^T with W stored [out][in] (no bias)."""
+    return f64(x) @ f64(w).T
+
+
+# ---------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------
+
+def attention(q, k, v, visible=None):
+    """Softmax attention per head, fp64, with max subtraction.
+
+    q: [N][H][D], k, v: [S][H][D]; visible: optional bool [N][S] (True = may
+    attend).  Scale 1/sqrt(D).  Returns [N][H][D].
+    """
+    q, k, v = f64(q), f64(k), f64(v)
+    n, h, d = q.shape
+    out = np.empty((n, h, d))
+    for hh in range(h):
+        logits = (q[:, hh, :] @ k[:, hh, :].T) / math.sqrt(d)
+        if visible is not None:
+            logits = np.where(visible, logits, -np.inf)
+        logits = logits - logits.max(axis=1, keepdims=True)
+        p = np.exp(logits)
+        p = p / p.sum(axis=1, keepdims=True)
+        out[:, hh, :] = p @ v[:, hh, :]
+    return out
+
+
+def block_causal_visible(q_units, k_units):
+    """Block-causal mask: a query in unit j sees every key whose unit is <= j
+    (bidirectional inside a unit) -- [v0.1] §3.3, [dig] "method overview"."""
+    return np.asarray(k_units)[None, :] <= np.asarray(q_units)[:, None]
+
+
+# ---------------------------------------------------------------------------
+# K/V cache (pre-allocated, ring of unit slots)
+# ---------------------------------------------------------------------------
+
+class KVCache:
+    """Pre-allocated per-layer K/V cache of n_slots unit slots of T_u tokens.
+
+    The thinker's K/V slice for unit u is written verbatim into slot
+    u mod n_slots ([dig] "performer path": each rank writes the broadcast slice
+    into its pre-allocated local cache).  Valid rows are the first
+    min(units, n_slots) * T_u rows.  With ring=False a full cache refuses the
+    append and stays unchanged.
+    """
+
+    def __init__(self, n_layers, n_slots, unit_tokens, n_heads, head_dim, ring=True, dtype=np.float64):
+        self.n_slots = n_slots
+        self.unit_tokens = unit_tokens
+        self.ring = ring
+        shape = (n_layers, n_slots * unit_tokens, n_heads, head_dim)
+        self.k = np.zeros(shape, dtype=dtype)
+        self.v = np.zeros(shape, dtype=dtype)
+        self.units = 0          # units ever appended (evicted ones included)
+
+    @property
+    def tokens_appended(self):
+        return self.units * self.unit_tokens
+
+    @property
+    def valid_tokens(self):
+        return min(self.units, self.n_slots) * self.unit_tokens
+
+    def append(self, k_slice, v_slice):
+        """k_slice, v_slice: [L][n_units * T_u][H][D].  Returns False (and changes
+        nothing) when the cache is full and ring is off."""
+        t = self.unit_tokens
+        n_tok = k_slice.shape[1]
+        if n_tok % t != 0:
+            raise ValueError("slice length must be a whole number of units")
+        n_units = n_tok // t
+        if not self.ring and self.units + n_units > self.n_slots:
+            return False
+        for i in range(n_units):
+            slot = (self.units + i) % self.n_slots
+            self.k[:, slot * t:(slot + 1) * t] = k_slice[:, i * t:(i + 1) * t]
+            self.v[:, slot * t:(slot + 1) * t] = v_slice[:, i * t:(i + 1) * t]
+        self.units += n_units
+        return True
+
+
+# ---------------------------------------------------------------------------
+# the velocity network f_theta (performer form)
+# ---------------------------------------------------------------------------
+
+def embed(cfg: Config, z, tau, w, modality=None):
+    """x_j = W_in z_j + e_mod[m(j)] + temb(tau).  Audio and video noisy latents
+    enter together ([v0.1] §3.4 cross-modal conditioning)."""
+    if modality is None:
+        modality = modality_of_tokens(cfg)
+    x = linear(z, w["w_in"])
+    x = x + f64(w["e_mod"])[modality]
+    x = x + tau_embedding(tau, cfg.d_model)[None, :]
+    return x
+
+
+def layer_forward(cfg: Config, x, lw, k_ctx, v_ctx, pos, visible=None, return_kv=False):
+    """One pre-norm block.  k_ctx/v_ctx: clean context keys/values [S][H][D]
+    (already rotated); the current tokens' own k, v are appended after them."""
+    n = x.shape[0]
+    h = rmsnorm(x, lw["g_attn"], cfg.rms_eps)
+    qkv = linear(h, lw["w_qkv"])
+    hd = cfg.hd
+    q = qkv[:, :hd].reshape(n, cfg.n_heads, cfg.head_dim)
+    k = qkv[:, hd:2 * hd].reshape(n, cfg.n_heads, cfg.head_dim)
+    v = qkv[:, 2 * hd:].reshape(n, cfg.n_heads, cfg.head_dim)
+    q = rope(q, pos, cfg.rope_theta)
+    k = rope(k, pos, cfg.rope_theta)
+    K = np.concatenate([f64(k_ctx), k], axis=0)
+    V = np.concatenate([f64(v_ctx), v], axis=0)
+    a = attention(q, K, V, visible)
+    x = x + linear(a.reshape(n, hd), lw["w_o"])
+    h2 = rmsnorm(x, lw["g_mlp"], cfg.rms_eps)
+    x = x + linear(gelu_tanh(linear(h2, lw["w_1"])), lw["w_2"])
+    if return_kv:
+        return x, k, v
+    return x
+
+
+def head(cfg: Config, x, w):
+    """Velocity head: v = RMSNorm(x; g_f) W_out^T, one C-vector per token."""
+    return linear(rmsnorm(x, w["g_final"], cfg.rms_eps), w["w_out"])
+
+
+def f_theta(cfg: Config, z, tau, w, cache_k, cache_v, valid_tokens, p0, pos=None, modality=None):
+    """Velocity of the current unit's noisy latents z [N][C] at flow time tau.
+
+    Performer form: every current-unit query sees every valid cached token
+    (all cached units precede the current one) and every current-unit token
+    (bidirectional inside the unit) -- [v0.1] §3.3 block-causal attention,
+    clean context c_k of §3.4.  cache_k/cache_v: per-layer [rows][H][D]; only
+    the first valid_tokens rows are context.  pos/modality override the
+    default token positions (p0 + j) and modality ids (video, then audio).
+    """
+    x = embed(cfg, z, tau, w, modality)
+    if pos is None:
+        pos = p0 + np.arange(cfg.n_tokens)
+    for li, lw in enumerate(w["layers"]):
+        kc = f64(cache_k[li][:valid_tokens])
+        vc = f64(cache_v[li][:valid_tokens])
+        x = layer_forward(cfg, x, lw, kc, vc, pos)
+    return head(cfg, x, w)
+
+
+def euler_step(z, v, tau_from, tau_to):
+    """One Euler step along the flow: z <- z + (tau_to - tau_from) v."""
+    return f64(z) + (float(tau_to) - float(tau_from)) * f64(v)
+
+
+def fm_solve(z, taus, velocity):
+    """Integrate dz/dtau = velocity(z, tau) from taus[0] (= 1, pure noise) to
+    taus[-1] (= 0, clean latent) with explicit Euler steps ([v0.1] §3.4: the
+    linear path has a constant velocity field, so few steps suffice)."""
+    z = f64(z)
+    for i in range(len(taus) - 1):
+        z = euler_step(z, velocity(z, taus[i]), taus[i], taus[i + 1])
+    return z
+
+
+def uniform_taus(n_steps):
+    """Uniform schedule 1 -> 0 in n_steps steps."""
+    return [1.0 - i / n_steps for i in range(n_steps + 1)]
+
+
+def rf_path(z0, eps, tau):
+    """Rectified-flow linear path z_tau = (1 - tau) z0 + tau eps."""
+    return (1.0 - tau) * f64(z0) + tau * f64(eps)
+
+
+def rf_velocity(z0, eps):
+    """Constant velocity of the linear path: d z_tau / d tau = eps - z0."""
+    return f64(eps) - f64(z0)
+
+
+def denoise_solve(cfg: Config, eps, taus, w, cache_k, cache_v, valid_tokens, p0):
+    """The performer's solve for one unit: Euler over f_theta from eps at tau=1."""
+    return fm_solve(eps, taus,
+                    lambda z, t: f_theta(cfg, z, t, w, cache_k, cache_v, valid_tokens, p0))
+
+
+# ---------------------------------------------------------------------------
+# block-causal full-sequence form (prefill / invariant checks)
+# ---------------------------------------------------------------------------
+
+def f_theta_sequence(cfg: Config, zs, taus, w, return_kv=False):
+    """Masked block-causal forward over several units at once.
+
+    zs: list of per-unit latents [N][C]; taus: per-unit flow times.  Token j of
+    unit u is at absolute position u * N + j and sees every token of units <= u.
+    Returns the per-unit velocities, and optionally every layer's rotated K/V
+    per unit (what a cache built from these units would hold).
+    """
+    n = cfg.n_tokens
+    n_units = len(zs)
+    x = np.concatenate([embed(cfg, zs[u], taus[u], w) for u in range(n_units)], axis=0)
+    units = np.repeat(np.arange(n_units), n)
+    pos = np.arange(n_units * n)
+    visible = block_causal_visible(units, units)
+    kv = []
+    empty = np.zeros((0, cfg.n_heads, cfg.head_dim))
+    for lw in w["layers"]:
+        x, k, v = layer_forward(cfg, x, lw, empty, empty, pos, visible, return_kv=True)
+        kv.append((k, v))
+    vel = head(cfg, x, w)
+    out = [vel[u * n:(u + 1) * n] for u in range(n_units)]
+    if return_kv:
+        return out, kv
+    return out
+
+
+# ---------------------------------------------------------------------------
+# work counts (for the timed CPU baseline)
+# ---------------------------------------------------------------------------
+
+def step_flops(cfg: Config, valid_tokens):
+    """Dense FLOPs of one f_theta evaluation: 2MKN per matmul, 4 N S H D for attention."""
+    n, d, hd, f = cfg.n_tokens, cfg.d_model, cfg.hd, cfg.d_mlp
+    gemm = 2 * n * d * (3 * hd) + 2 * n * hd * d + 2 * n * d * f + 2 * n * f * d
+    attn = 4 * n * (valid_tokens + n) * hd
+    return cfg.n_layers * (gemm + attn) + 2 * n * cfg.c_lat * d * 2

@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark: the performer's next-unit denoise of a 640x368 unit on B200.
+
+One bench step = one pass of the whole hot path for one unit: the thinker's
+1200-token K/V slice is appended to the session's 48-unit ring cache (evicting
+the oldest unit, so 57,600 cached tokens stay valid), then the 924 latent
+tokens (920 video + 4 audio) are solved from noise with 4 Euler steps of the
+28-layer velocity network.  Inputs are synthetic (seeded), resident in HBM and
+far larger than L2 (6.3 GB of weights + 19.8 GB of cache are read per Euler
+step), so no L2 flush is needed between steps.
+
+value = Euler denoise steps per second summed over all ranks (each rank runs
+its own session: weak scaling, no collective on the data path).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "640x368 unit denoise steps/s"
+UNIT = "denoise steps/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="v0.2-640x368")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16": p["bf16_tflops"],
+                "bf16_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--id={self.index}", "--query-gpu=" + ",".join(self.FIELDS),
+               "--format=csv,noheader,nounits", "-lms", "200"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[3:]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# work counts
+# ---------------------------------------------------------------------------
+def flop_counts(w, valid):
+    n, d, hd, f, L = w.n_tokens, w.d_model, w.hd, w.d_mlp, w.n_layers
+    attn = 4 * n * (valid + n) * hd
+    gemm = 2 * n * d * 3 * hd + 2 * n * hd * d + 2 * n * d * f + 2 * n * f * d
+    return {"attention_per_launch": attn, "gemm_per_layer": gemm,
+            "per_euler_step": L * (attn + gemm)}
+
+
+def append_bytes(w):
+    return 2 * 2 * w.n_layers * w.unit_kv_tokens * w.hd * 2   # K and V, read + write, bf16
+
+
+def source_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_for(kernel_src):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        ent = t[os.path.basename(kernel_src)]
+        if ent["source_sha256_16"] != source_hash(kernel_src):
+            return None
+        return ent["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the same workload
+# ---------------------------------------------------------------------------
+def cpu_sample(w, budget_s):
+    """Time the oracle's f_theta at the bench shapes on a bounded sample: the
+    embedding, as many of the 28 layers as fit the budget (each over the full
+    57,600-token cache), and the head; extrapolate to one Euler step."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_info
+
+    import sfm_synth as S
+    from oracle import sfm_oracle as O
+
+    cfg = O.Config(w.n_layers, w.d_model, w.n_heads, w.head_dim, w.d_mlp, w.c_lat, w.n_video,
+                   w.n_audio, w.unit_kv_tokens, w.rope_theta, w.rms_eps)
+    one = w.replace(n_layers=1)
+    weights = S.make_weights(one)
+    k, v = S.make_kv_slices(one, w.cache_units)
+    _, eps = S.make_latents(w)
+    valid = w.cache_units * w.unit_kv_tokens
+    kc, vc = O.f64(k[0]), O.f64(v[0])
+    lw = {n: O.f64(t) for n, t in weights["layers"][0].items()}
+    t0 = time.perf_counter()
+    x = O.embed(cfg, eps[0], 1.0, weights)
+    t_embed = time.perf_counter() - t0
+    pos = valid + np.arange(w.n_tokens)
+    layer_times = []
+    t_start = time.perf_counter()
+    while not layer_times or (time.perf_counter() - t_start < budget_s and len(layer_times) < w.n_layers):
+        t0 = time.perf_counter()
+        x = O.layer_forward(cfg, x, lw, kc, vc, pos)
+        layer_times.append(time.perf_counter() - t0)
+    t0 = time.perf_counter()
+    O.head(cfg, x, weights)
+    t_head = time.perf_counter() - t0
+    t_step = t_embed + w.n_layers * statistics.mean(layer_times) + t_head
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    sample = (f"oracle f_theta (numpy fp64) at the {w.name} unit over the full {valid}-token cache: "
+              f"embed + {len(layer_times)} of {w.n_layers} layers + head timed, "
+              f"x{w.n_layers}/{len(layer_times)} layers extrapolated to one Euler step")
+    del torch
+    return t_step, threads, sample
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    budget = max(1.0, min(args.cpu_budget_s, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_sample(w, budget)
+    times = []
+    for _ in range(args.steps):
+        t, threads, sample = cpu_sample(w, budget)
+        times.append(t)
+    t_step = statistics.mean(times)
+    value = 1.0 / t_step
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_step * 1e3 * w.n_steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": config_of(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    return {"workload": f"{w.name} unit: kvcache_append of one {w.unit_kv_tokens}-token slice + "
+                        f"{w.n_steps}-step Euler solve",
+            "tokens_per_unit": w.n_tokens, "video_tokens": w.n_video, "audio_tokens": w.n_audio,
+            "cache_tokens": w.cache_units * w.unit_kv_tokens, "layers": w.n_layers,
+            "d_model": w.d_model, "heads": w.n_heads, "head_dim": w.head_dim, "d_mlp": w.d_mlp,
+            "euler_steps": w.n_steps, "parallelism": "one session per GPU, no collectives",
+            "l2": "inputs larger than L2 (weights + cache read every Euler step)"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import sfm_synth as S
+    from streaming_flow_matching_b200 import Performer, _lib as L
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    weights = S.make_weights(w, device=dev)
+    p = Performer.from_workload(w, weights)
+    s = p.open_session(w.cache_units)
+    k, v = S.make_kv_slices(w, w.cache_units, device=dev)
+    p.kvcache_append(s, k, v)
+    del k, v
+    g = torch.Generator(device=dev)
+    g.manual_seed(11 + rank)
+    shape = (w.n_layers, w.unit_kv_tokens, w.n_heads, w.head_dim)
+    k1 = torch.randn(*shape, generator=g, device=dev).to(torch.bfloat16)
+    v1 = torch.randn(*shape, generator=g, device=dev).to(torch.bfloat16)
+    _, eps = S.make_latents(w, device=dev)
+    eps = eps[0].contiguous()
+    z = eps.clone()
+    taus = S.uniform_taus(w.n_steps)
+    torch.cuda.synchronize()
+
+    def step():
+        p.kvcache_append(s, k1, v1)
+        z.copy_(eps)
+        p.fm_solve(s, z, taus)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.4)
+    n0 = L.lib.sfm_kernel_launch_count()
+    L.profile_begin(1 << 16)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    prof = L.profile_end()
+    launches = L.lib.sfm_kernel_launch_count() - n0
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = t.item()
+    barrier()
+
+    # end to end: host (pinned) inputs copied in and the latents copied out every step
+    e2e = None
+    if not args.no_e2e:
+        k1_h = k1.cpu().pin_memory()
+        v1_h = v1.cpu().pin_memory()
+        eps_h = eps.cpu().pin_memory()
+        z_h = torch.empty_like(eps_h).pin_memory()
+
+        def e2e_step():
+            k1.copy_(k1_h, non_blocking=True)
+            v1.copy_(v1_h, non_blocking=True)
+            z.copy_(eps_h, non_blocking=True)
+            p.kvcache_append(s, k1, v1)
+            p.fm_solve(s, z, taus)
+            z_h.copy_(z, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = k1.numel() * 2 + v1.numel() * 2 + eps.numel() * 4
+        e2e = {"value": w.n_steps * args.steps * world / (te.item() / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": z.numel() * 4}
+        barrier()
+
+    if rank == 0:
+        pk = peaks()
+        valid = w.cache_units * w.unit_kv_tokens
+        fl = flop_counts(w, valid)
+        a_ms, a_n = prof["attention"]
+        attn_avg_ms = a_ms / max(a_n, 1)
+        attn_tflops = fl["attention_per_launch"] / (attn_avg_ms / 1e3) / 1e12
+        gemm_ms = sum(prof[k][0] for k in ("gemm_qkv", "gemm_o", "gemm_up", "gemm_down"))
+        contraction_ms = a_ms + prof["attention_merge"][0] + gemm_ms
+        contraction_flop = args.steps * w.n_steps * fl["per_euler_step"]
+        ap_ms, ap_n = prof["append"]
+        append_gbs = append_bytes(w) / (ap_ms / max(ap_n, 1) / 1e3) / 1e9 if ap_n else None
+        attn_src = os.path.join(ROOT, "streaming_flow_matching_b200", "csrc", "attn_simt.cu")
+        traffic = traffic_for(attn_src)
+        unit_ms = ms_max / args.steps
+        line = {
+            "metric": METRIC,
+            "value": w.n_steps * args.steps * world / (ms_max / 1e3),
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": unit_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded), resident in HBM",
+            "config": config_of(w),
+            "unit_latency_ms": unit_ms,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "roofline": {"kernel": "attention (flash, split-KV)", "bound": "tensor",
+                         "achieved": attn_tflops, "peak": pk["bf16_sustained"],
+                         "unit": "TFLOP/s", "frac": attn_tflops / pk["bf16_sustained"],
+                         "traffic": traffic,
+                         "peak_note": f"{pk['source']} sustained bf16 (kernel timed inside a long step)",
+                         "flop_per_launch": fl["attention_per_launch"],
+                         "avg_launch_ms": attn_avg_ms},
+            "contractions": {"tflops": contraction_flop / (contraction_ms / 1e3) / 1e12,
+                             "frac_of_bf16_peak": contraction_flop / (contraction_ms / 1e3) / 1e12
+                             / pk["bf16_sustained"],
+                             "attn_gemm_device_ms_per_unit": contraction_ms / args.steps},
+            "append": {"gb_s": append_gbs, "frac_of_hbm": (append_gbs / pk["hbm_gbs"]) if append_gbs else None,
+                       "bytes": append_bytes(w)},
+            "kernel_ms_per_unit": {k2: round(v2[0] / args.steps, 4) for k2, v2 in prof.items()},
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            t_step, threads, sample = cpu_sample(w, args.cpu_budget_s)
+            line["cpu_baseline"] = {"value": 1.0 / t_step, "unit": UNIT, "cores": threads,
+                                    "kind": "oracle", "sample": sample}
+        print(json.dumps(line), flush=True)
+    p.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    import sfm_synth as S
+    w = S.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

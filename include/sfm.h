@@ -35,6 +35,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define SFM_API __attribute__((visibility("default")))
+#else
+#define SFM_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -58,10 +64,10 @@ typedef struct sfm_handle sfm_handle;   /* opaque, library-owned */
 /* Shapes of f_theta and of one streaming unit. */
 typedef struct sfm_config {
   int n_layers;          /* L                                                   */
-  int d_model;           /* d: multiple of 64                                   */
+  int d_model;           /* d: multiple of 128 (bf16) / 64 (fp32)               */
   int n_heads;           /* H                                                   */
-  int head_dim;          /* D_h: 128 for bf16; even and <= 128 for fp32         */
-  int d_mlp;             /* F: multiple of 64                                   */
+  int head_dim;          /* D_h: 128 for bf16; a multiple of 32, <= 128 for fp32 */
+  int d_mlp;             /* F: multiple of 128 (bf16) / 64 (fp32)               */
   int c_lat;             /* C: latent channels per token (<= 64)                */
   int n_video;           /* video tokens of the current unit (raster order)     */
   int n_audio;           /* audio tokens of the current unit (after the video)  */
@@ -120,20 +126,20 @@ typedef struct sfm_session_info {
  * elements) and all scratch on the current device.  Returns SFM_EINVAL /
  * SFM_EUNSUPPORTED for bad shapes, SFM_ENOMEM if allocation fails.  The hot
  * path allocates nothing after this call. */
-int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out);
+SFM_API int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out);
 
 /* Frees everything the handle owns (synchronises the device first). */
-void sfm_destroy(sfm_handle* h);
+SFM_API void sfm_destroy(sfm_handle* h);
 
 /* Carves a contiguous cache region of cache_units unit slots (plus the
  * current unit's scratch rows) out of the pool for a new session.
  * SFM_ECAPACITY if the pool or the session table is full. */
-int sfm_session_open(sfm_handle* h, int cache_units, int* session);
+SFM_API int sfm_session_open(sfm_handle* h, int cache_units, int* session);
 
 /* Forgets a session's units (counters to zero); its region stays reserved. */
-int sfm_session_reset(sfm_handle* h, int session);
+SFM_API int sfm_session_reset(sfm_handle* h, int session);
 
-int sfm_session_get_info(const sfm_handle* h, int session, sfm_session_info* out);
+SFM_API int sfm_session_get_info(const sfm_handle* h, int session, sfm_session_info* out);
 
 /* ---- the hot path ------------------------------------------------------- */
 
@@ -145,13 +151,13 @@ int sfm_session_get_info(const sfm_handle* h, int session, sfm_session_info* out
  * SFM_EINVAL if n_tok is not a positive multiple of T_u; SFM_ECAPACITY if
  * ring == 0 and the units do not fit (nothing is written).
  */
-int sfm_kvcache_append(sfm_handle* h, int session, const void* k, const void* v,
+SFM_API int sfm_kvcache_append(sfm_handle* h, int session, const void* k, const void* v,
                        int n_tok, void* stream);
 
 /* Copies cache rows [row0, row0 + n_rows) of one layer into caller device
  * buffers k_dst, v_dst ([n_rows][H][D_h]).  Rows index the session's region
  * (slot s occupies rows [s T_u, (s+1) T_u)). */
-int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long long row0,
+SFM_API int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long long row0,
                      long long n_rows, void* k_dst, void* v_dst, void* stream);
 
 /*
@@ -160,7 +166,7 @@ int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long long row0
  * n_audio (video rows first), updated in place.  v_out: nullable device fp32
  * [N][C] receiving v.  The current unit's tokens are at positions p0 + j.
  */
-int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_from,
+SFM_API int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_from,
                      float tau_to, float* v_out, void* stream);
 
 /*
@@ -169,13 +175,13 @@ int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_from,
  * taus[n-1] = 0 (z then holds the unit's clean latent).  The cache is not
  * modified (the current unit's K/V are scratch, never committed).
  */
-int sfm_fm_solve(sfm_handle* h, int session, float* z, const float* taus,
+SFM_API int sfm_fm_solve(sfm_handle* h, int session, float* z, const float* taus,
                  int n_taus, void* stream);
 
 /* Batched solve over n_sessions open sessions (distinct ids), each with its
  * own cache length; z[i] is session i's device fp32 [N][C].  sessions and z
  * are host arrays.  SFM_ECAPACITY if n_sessions > max_sessions. */
-int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions,
+SFM_API int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions,
                          float* const* z, const float* taus, int n_taus, void* stream);
 
 /* ---- standalone kernels --------------------------------------------------- */
@@ -189,19 +195,44 @@ int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions,
  * sfm_attention_workspace_bytes(...) bytes (caller-owned; may be NULL when
  * that size is 0).  n_kv >= 1.
  */
-size_t sfm_attention_workspace_bytes(int n_q, int n_kv, int n_heads, int head_dim, int dtype);
-int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q, int n_kv,
+SFM_API size_t sfm_attention_workspace_bytes(int n_q, int n_kv, int n_heads, int head_dim, int dtype);
+SFM_API int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q, int n_kv,
                   int n_heads, int head_dim, int dtype, void* workspace,
                   size_t workspace_bytes, void* stream);
 
 /* Vectorised Euler update z[i] += dtau * v[i], i < n; device fp32. */
-int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream);
+SFM_API int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream);
+
+/* ---- measurement ------------------------------------------------------------ */
+/* Kernel classes timed by the profiler (index into the arrays below). */
+#define SFM_PROF_APPEND     0   /* K/V cache append                          */
+#define SFM_PROF_ATTN       1   /* attention (flash kernel)                  */
+#define SFM_PROF_ATTN_MERGE 2   /* split-KV merge                            */
+#define SFM_PROF_GEMM_QKV   3   /* QKV projection                            */
+#define SFM_PROF_GEMM_O     4   /* O projection + residual                   */
+#define SFM_PROF_GEMM_UP    5   /* MLP up + GELU                             */
+#define SFM_PROF_GEMM_DOWN  6   /* MLP down + residual                       */
+#define SFM_PROF_ROWOPS     7   /* embed, RMSNorm, RoPE, scatter, tables     */
+#define SFM_PROF_HEAD       8   /* velocity head + Euler update              */
+#define SFM_PROF_KINDS      9
+
+/* Starts recording a CUDA event pair around every kernel this library
+ * launches on this host thread (events on the launching stream), for up to
+ * max_launches launches; later launches are not recorded.  Allocates the
+ * events (not on the hot path).  SFM_EINVAL if max_launches < 1. */
+SFM_API int sfm_profile_begin(int max_launches);
+/* Synchronises the recorded events, stops recording and returns, per kernel
+ * class, the summed device time in ms and the launch count (host arrays of
+ * SFM_PROF_KINDS entries). */
+SFM_API int sfm_profile_end(double* ms, long long* launches);
+/* Kernels launched by this library in this process so far. */
+SFM_API unsigned long long sfm_kernel_launch_count(void);
 
 /* ---- errors --------------------------------------------------------------- */
-const char* sfm_strerror(int status);
+SFM_API const char* sfm_strerror(int status);
 /* The cudaError_t of the last failed CUDA call made by this library on this
  * host thread (0 if none). */
-int sfm_last_cuda_error(void);
+SFM_API int sfm_last_cuda_error(void);
 
 #ifdef __cplusplus
 }

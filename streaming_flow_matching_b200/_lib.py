@@ -1,0 +1,113 @@
+"""ctypes declarations of libsfm's C ABI (include/sfm.h), same names and arguments.
+
+Loading fails loudly when the library has not been built: there is no other
+implementation of these calls in this package.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsfm.so")
+
+SFM_OK, SFM_EINVAL, SFM_ECAPACITY, SFM_ESESSION, SFM_ECUDA, SFM_ENOMEM, SFM_EUNSUPPORTED = (
+    0, -1, -2, -3, -4, -5, -6)
+SFM_DTYPE_BF16, SFM_DTYPE_FP32 = 0, 1
+
+
+class sfm_config(C.Structure):
+    _fields_ = [("n_layers", C.c_int), ("d_model", C.c_int), ("n_heads", C.c_int),
+                ("head_dim", C.c_int), ("d_mlp", C.c_int), ("c_lat", C.c_int),
+                ("n_video", C.c_int), ("n_audio", C.c_int), ("unit_kv_tokens", C.c_int),
+                ("max_sessions", C.c_int), ("pool_tokens", C.c_longlong), ("dtype", C.c_int),
+                ("ring", C.c_int), ("rope_theta", C.c_double), ("rms_eps", C.c_double)]
+
+
+_PP = C.POINTER(C.c_void_p)
+
+
+class sfm_weights(C.Structure):
+    _fields_ = [("w_in", C.c_void_p), ("e_mod", C.c_void_p), ("g_final", C.c_void_p),
+                ("w_out", C.c_void_p), ("g_attn", _PP), ("w_qkv", _PP), ("w_o", _PP),
+                ("g_mlp", _PP), ("w_1", _PP), ("w_2", _PP)]
+
+
+class sfm_session_info(C.Structure):
+    _fields_ = [("cache_units", C.c_int), ("units_appended", C.c_longlong),
+                ("valid_tokens", C.c_longlong), ("p0", C.c_longlong), ("base_row", C.c_longlong)]
+
+
+class SfmError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        msg = lib.sfm_strerror(status).decode() if lib is not None else str(status)
+        if status == SFM_ECUDA:
+            msg += f" (cudaError {lib.sfm_last_cuda_error()})"
+        super().__init__(f"{what}: {msg} [{status}]" if what else f"{msg} [{status}]")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libsfm.so is not built ({LIB_PATH}); build it with "
+            "`python -m streaming_flow_matching_b200.build`")
+    L = C.CDLL(LIB_PATH)
+    vp, i, ll, f, sz = C.c_void_p, C.c_int, C.c_longlong, C.c_float, C.c_size_t
+    sig = {
+        "sfm_create": (i, [C.POINTER(sfm_config), C.POINTER(sfm_weights), C.POINTER(vp)]),
+        "sfm_destroy": (None, [vp]),
+        "sfm_session_open": (i, [vp, i, C.POINTER(i)]),
+        "sfm_session_reset": (i, [vp, i]),
+        "sfm_session_get_info": (i, [vp, i, C.POINTER(sfm_session_info)]),
+        "sfm_kvcache_append": (i, [vp, i, vp, vp, i, vp]),
+        "sfm_kvcache_read": (i, [vp, i, i, ll, ll, vp, vp, vp]),
+        "sfm_denoise_step": (i, [vp, i, vp, f, f, vp, vp]),
+        "sfm_fm_solve": (i, [vp, i, vp, C.POINTER(f), i, vp]),
+        "sfm_fm_solve_batched": (i, [vp, i, C.POINTER(i), C.POINTER(vp), C.POINTER(f), i, vp]),
+        "sfm_attention_workspace_bytes": (sz, [i, i, i, i, i]),
+        "sfm_attention": (i, [vp, vp, vp, vp, i, i, i, i, i, vp, sz, vp]),
+        "sfm_euler_update": (i, [vp, vp, f, ll, vp]),
+        "sfm_profile_begin": (i, [i]),
+        "sfm_profile_end": (i, [C.POINTER(C.c_double), C.POINTER(ll)]),
+        "sfm_kernel_launch_count": (C.c_ulonglong, []),
+        "sfm_strerror": (C.c_char_p, [i]),
+        "sfm_last_cuda_error": (i, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+lib = None
+lib = _load()
+
+# Every symbol declared in include/sfm.h, in declaration order.
+EXPORTS = ["sfm_create", "sfm_destroy", "sfm_session_open", "sfm_session_reset",
+           "sfm_session_get_info", "sfm_kvcache_append", "sfm_kvcache_read", "sfm_denoise_step",
+           "sfm_fm_solve", "sfm_fm_solve_batched", "sfm_attention_workspace_bytes",
+           "sfm_attention", "sfm_euler_update", "sfm_profile_begin", "sfm_profile_end",
+           "sfm_kernel_launch_count", "sfm_strerror", "sfm_last_cuda_error"]
+
+PROF_KINDS = ["append", "attention", "attention_merge", "gemm_qkv", "gemm_o", "gemm_up",
+              "gemm_down", "rowops", "head_euler"]
+
+
+def profile_begin(max_launches=1 << 16):
+    check(lib.sfm_profile_begin(max_launches), "sfm_profile_begin")
+
+
+def profile_end():
+    """Per kernel class: (summed device ms, launches) since profile_begin."""
+    ms = (C.c_double * len(PROF_KINDS))()
+    n = (C.c_longlong * len(PROF_KINDS))()
+    check(lib.sfm_profile_end(ms, n), "sfm_profile_end")
+    return {k: (ms[i], n[i]) for i, k in enumerate(PROF_KINDS)}
+
+
+def check(status, what=""):
+    if status != SFM_OK:
+        raise SfmError(status, what)
+    return status

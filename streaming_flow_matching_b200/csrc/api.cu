@@ -1,0 +1,479 @@
+// C ABI of libsfm: argument validation, ownership of the K/V pool and the
+// scratch activations, session bookkeeping, and the per-step launch sequence
+// of f_theta.  Every error is caught on the host before any launch.
+#include <math.h>
+#include <string.h>
+
+#include <new>
+
+#include "attn.cuh"
+#include "common.cuh"
+
+using namespace sfm;
+
+namespace sfm {
+static thread_local int g_last_cuda_error = 0;
+
+int record_cuda(cudaError_t e) {
+  count_launch();
+  if (e == cudaSuccess) return SFM_OK;
+  g_last_cuda_error = (int)e;
+  return SFM_ECUDA;
+}
+}  // namespace sfm
+
+struct sfm_handle {
+  sfm_config cfg{};
+  int n_tok = 0;
+  int es = 2;                    // bytes per stored element
+  int hd = 0;                    // H * D_h
+  bool has_weights = false;
+  const void *w_in = nullptr, *e_mod = nullptr, *g_final = nullptr, *w_out = nullptr;
+  std::vector<const void*> g_attn, w_qkv, w_o, g_mlp, w_1, w_2;
+  void* k_pool = nullptr;
+  void* v_pool = nullptr;
+  long long pool_used = 0;
+  std::vector<Session> sessions;
+  // scratch, sized for max_sessions * n_tok rows
+  float* x = nullptr;        // [M][d] fp32 residual stream
+  void* xn = nullptr;        // [M][d] normalised GEMM operand
+  float* qkv32 = nullptr;    // [M][3 H D] fp32 projection output
+  void* q = nullptr;         // [M][H][D] rotated queries
+  void* ao = nullptr;        // [M][H D] attention output
+  void* hmlp = nullptr;      // [M][F] GELU(MLP-up)
+  float* cos_t = nullptr;    // [M][D/2]
+  float* sin_t = nullptr;
+  float* o_part = nullptr;   // [kMaxSplits][M][H][D]
+  float* lse_part = nullptr; // [kMaxSplits][M][H]
+  std::vector<void*> owned;
+
+  void* layer_k(int l) const { return (char*)k_pool + (size_t)l * cfg.pool_tokens * hd * es; }
+  void* layer_v(int l) const { return (char*)v_pool + (size_t)l * cfg.pool_tokens * hd * es; }
+};
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+int validate_config(const sfm_config* c) {
+  if (!c) return SFM_EINVAL;
+  if (c->n_layers < 1 || c->d_model < 1 || c->n_heads < 1 || c->head_dim < 1 || c->d_mlp < 1 ||
+      c->c_lat < 1 || c->n_video < 0 || c->n_audio < 0 || c->n_video + c->n_audio < 1 ||
+      c->unit_kv_tokens < 1 || c->max_sessions < 1 || c->pool_tokens < 0)
+    return SFM_EINVAL;
+  if (c->dtype != SFM_DTYPE_BF16 && c->dtype != SFM_DTYPE_FP32) return SFM_EINVAL;
+  if (!(c->rms_eps >= 0.0) || !(c->rope_theta > 0.0)) return SFM_EINVAL;
+  if (c->max_sessions > kMaxBatch) return SFM_EUNSUPPORTED;
+  if (c->c_lat > 64 || c->d_model % 2) return SFM_EUNSUPPORTED;
+  const int hd = c->n_heads * c->head_dim;
+  if (c->dtype == SFM_DTYPE_BF16) {
+    // GEMM tiles: N in multiples of 128, K in multiples of 64; flash tiles: D_h = 128
+    if (c->head_dim != 128 || c->d_model % 128 || c->d_mlp % 128 || (3 * hd) % 128 || hd % 64)
+      return SFM_EUNSUPPORTED;
+  } else {
+    if (c->head_dim % 32 || c->head_dim > 128 || c->d_model % 64 || c->d_mlp % 64 ||
+        (3 * hd) % 64 || hd % 16)
+      return SFM_EUNSUPPORTED;
+  }
+  return SFM_OK;
+}
+
+template <typename T>
+int dalloc(sfm_handle* h, T** p, size_t bytes) {
+  void* q = nullptr;
+  if (bytes == 0) bytes = 16;
+  if (cudaMalloc(&q, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return SFM_ENOMEM;
+  }
+  h->owned.push_back(q);
+  *p = (T*)q;
+  return SFM_OK;
+}
+
+int session_ok(const sfm_handle* h, int s) {
+  if (!h) return SFM_EINVAL;
+  if (s < 0 || s >= (int)h->sessions.size() || !h->sessions[s].open) return SFM_ESESSION;
+  return SFM_OK;
+}
+
+long long valid_tokens(const sfm_handle* h, const Session& s) {
+  const long long u = s.units < s.cache_units ? s.units : s.cache_units;
+  return u * h->cfg.unit_kv_tokens;
+}
+
+int fill_batch(const sfm_handle* h, int n, const int* sessions, BatchDesc* b) {
+  memset(b, 0, sizeof(*b));
+  b->n = n;
+  b->n_tok = h->n_tok;
+  b->n_video = h->cfg.n_video;
+  for (int i = 0; i < n; ++i) {
+    const Session& s = h->sessions[sessions[i]];
+    b->base[i] = s.base_row;
+    b->valid[i] = (int)valid_tokens(h, s);
+    b->p0[i] = s.units * h->cfg.unit_kv_tokens;
+  }
+  return SFM_OK;
+}
+
+AttnDesc attn_desc(const BatchDesc& b) {
+  AttnDesc a{};
+  a.n = b.n;
+  a.rows_per = b.n_tok;
+  for (int i = 0; i < b.n; ++i) {
+    a.kbase[i] = b.base[i];
+    a.nkeys[i] = b.valid[i] + b.n_tok;
+  }
+  return a;
+}
+
+// One Euler step of f_theta for the sessions in b (RoPE table already filled).
+int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from, float tau_to,
+             float* const* v_out, cudaStream_t s) {
+  const sfm_config& c = h->cfg;
+  const int M = b.n * b.n_tok;
+  const int d = c.d_model, hd = h->hd, F = c.d_mlp, dt = c.dtype;
+  const float eps = (float)c.rms_eps;
+  int rc;
+#define SFM_TRY(call) \
+  if ((rc = (call)) != SFM_OK) return rc;
+  {
+    ProfScope ps(SFM_PROF_ROWOPS, s);
+    SFM_TRY(launch_embed(b, z, h->w_in, h->e_mod, tau_from, h->x, d, c.c_lat, dt, s));
+  }
+  const AttnDesc ad = attn_desc(b);
+  long long max_keys = 0;
+  for (int i = 0; i < b.n; ++i) max_keys = ad.nkeys[i] > max_keys ? ad.nkeys[i] : max_keys;
+  const int splits = dt == SFM_DTYPE_BF16 ? attention_splits(b.n_tok, b.n, max_keys, c.n_heads) : 1;
+  for (int l = 0; l < c.n_layers; ++l) {
+    {
+      ProfScope ps(SFM_PROF_ROWOPS, s);
+      SFM_TRY(launch_rmsnorm(h->x, h->g_attn[l], h->xn, M, d, eps, dt, s));
+    }
+    {
+      ProfScope ps(SFM_PROF_GEMM_QKV, s);
+      SFM_TRY(launch_gemm(h->xn, h->w_qkv[l], h->qkv32, M, 3 * hd, d, EPI_F32, dt, s));
+    }
+    {
+      ProfScope ps(SFM_PROF_ROWOPS, s);
+      SFM_TRY(launch_rope_scatter(b, h->qkv32, h->cos_t, h->sin_t, h->q, h->layer_k(l),
+                                  h->layer_v(l), c.n_heads, c.head_dim, dt, s));
+    }
+    SFM_TRY(launch_attention(ad, h->q, h->layer_k(l), h->layer_v(l), h->ao, c.n_heads,
+                             c.head_dim, dt, splits, h->o_part, h->lse_part, s));
+    {
+      ProfScope ps(SFM_PROF_GEMM_O, s);
+      SFM_TRY(launch_gemm(h->ao, h->w_o[l], h->x, M, d, hd, EPI_RESID, dt, s));
+    }
+    {
+      ProfScope ps(SFM_PROF_ROWOPS, s);
+      SFM_TRY(launch_rmsnorm(h->x, h->g_mlp[l], h->xn, M, d, eps, dt, s));
+    }
+    {
+      ProfScope ps(SFM_PROF_GEMM_UP, s);
+      SFM_TRY(launch_gemm(h->xn, h->w_1[l], h->hmlp, M, F, d, EPI_GELU, dt, s));
+    }
+    {
+      ProfScope ps(SFM_PROF_GEMM_DOWN, s);
+      SFM_TRY(launch_gemm(h->hmlp, h->w_2[l], h->x, M, d, F, EPI_RESID, dt, s));
+    }
+  }
+  {
+    ProfScope ps(SFM_PROF_HEAD, s);
+    SFM_TRY(launch_head_euler(b, h->x, h->g_final, h->w_out, z, v_out, tau_to - tau_from, d,
+                              c.c_lat, eps, dt, s));
+  }
+#undef SFM_TRY
+  return SFM_OK;
+}
+
+int check_taus(const float* taus, int n_taus) {
+  if (!taus || n_taus < 2) return SFM_EINVAL;
+  for (int i = 0; i < n_taus; ++i)
+    if (!isfinite(taus[i])) return SFM_EINVAL;
+  return SFM_OK;
+}
+
+int solve(sfm_handle* h, int n, const int* sessions, float* const* z, const float* taus,
+          int n_taus, float* const* v_out, cudaStream_t s) {
+  BatchDesc b;
+  fill_batch(h, n, sessions, &b);
+  int rc;
+  {
+    ProfScope ps(SFM_PROF_ROWOPS, s);
+    rc = launch_rope_table(b, h->cos_t, h->sin_t, h->cfg.head_dim, h->cfg.rope_theta, s);
+  }
+  if (rc) return rc;
+  for (int i = 0; i + 1 < n_taus; ++i) {
+    rc = run_step(h, b, z, taus[i], taus[i + 1], v_out, s);
+    if (rc) return rc;
+  }
+  return SFM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
+  if (!out) return SFM_EINVAL;
+  *out = nullptr;
+  int rc = validate_config(cfg);
+  if (rc) return rc;
+  sfm_handle* h = new (std::nothrow) sfm_handle();
+  if (!h) return SFM_ENOMEM;
+  h->cfg = *cfg;
+  h->n_tok = cfg->n_video + cfg->n_audio;
+  h->es = cfg->dtype == SFM_DTYPE_BF16 ? 2 : 4;
+  h->hd = cfg->n_heads * cfg->head_dim;
+  if (((long long)h->hd * h->es) % 16) {
+    delete h;
+    return SFM_EUNSUPPORTED;
+  }
+  if (w) {
+    const void* const* arrays[6] = {w->g_attn, w->w_qkv, w->w_o, w->g_mlp, w->w_1, w->w_2};
+    if (!w->w_in || !w->e_mod || !w->g_final || !w->w_out) rc = SFM_EINVAL;
+    for (int a = 0; a < 6 && !rc; ++a) {
+      if (!arrays[a]) rc = SFM_EINVAL;
+      for (int l = 0; l < cfg->n_layers && !rc; ++l)
+        if (!arrays[a][l] || !aligned16(arrays[a][l])) rc = SFM_EINVAL;
+    }
+    if (rc) {
+      delete h;
+      return rc;
+    }
+    h->has_weights = true;
+    h->w_in = w->w_in;
+    h->e_mod = w->e_mod;
+    h->g_final = w->g_final;
+    h->w_out = w->w_out;
+    h->g_attn.assign(w->g_attn, w->g_attn + cfg->n_layers);
+    h->w_qkv.assign(w->w_qkv, w->w_qkv + cfg->n_layers);
+    h->w_o.assign(w->w_o, w->w_o + cfg->n_layers);
+    h->g_mlp.assign(w->g_mlp, w->g_mlp + cfg->n_layers);
+    h->w_1.assign(w->w_1, w->w_1 + cfg->n_layers);
+    h->w_2.assign(w->w_2, w->w_2 + cfg->n_layers);
+  }
+  h->sessions.resize(cfg->max_sessions);
+  const size_t L = cfg->n_layers, es = h->es, hd = h->hd;
+  const size_t M = (size_t)cfg->max_sessions * h->n_tok;
+  const size_t d = cfg->d_model, F = cfg->d_mlp;
+  const size_t pool_bytes = L * (size_t)cfg->pool_tokens * hd * es;
+  rc = dalloc(h, &h->k_pool, pool_bytes);
+  if (!rc) rc = dalloc(h, &h->v_pool, pool_bytes);
+  if (!rc && h->has_weights) {
+    if (!rc) rc = dalloc(h, &h->x, M * d * 4);
+    if (!rc) rc = dalloc(h, &h->xn, M * d * es);
+    if (!rc) rc = dalloc(h, &h->qkv32, M * 3 * hd * 4);
+    if (!rc) rc = dalloc(h, &h->q, M * hd * es);
+    if (!rc) rc = dalloc(h, &h->ao, M * hd * es);
+    if (!rc) rc = dalloc(h, &h->hmlp, M * F * es);
+    if (!rc) rc = dalloc(h, &h->cos_t, M * (cfg->head_dim / 2) * 4);
+    if (!rc) rc = dalloc(h, &h->sin_t, M * (cfg->head_dim / 2) * 4);
+    if (!rc && cfg->dtype == SFM_DTYPE_BF16) {
+      rc = dalloc(h, &h->o_part, (size_t)kMaxSplits * M * hd * 4);
+      if (!rc) rc = dalloc(h, &h->lse_part, (size_t)kMaxSplits * M * cfg->n_heads * 4);
+    }
+  }
+  if (rc) {
+    sfm_destroy(h);
+    return rc;
+  }
+  *out = h;
+  return SFM_OK;
+}
+
+void sfm_destroy(sfm_handle* h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  for (void* p : h->owned) cudaFree(p);
+  delete h;
+}
+
+int sfm_session_open(sfm_handle* h, int cache_units, int* session) {
+  if (!h || !session || cache_units < 1) return SFM_EINVAL;
+  int slot = -1;
+  for (int i = 0; i < (int)h->sessions.size(); ++i)
+    if (!h->sessions[i].open) {
+      slot = i;
+      break;
+    }
+  if (slot < 0) return SFM_ECAPACITY;
+  const long long rows = (long long)cache_units * h->cfg.unit_kv_tokens + h->n_tok;
+  if (h->pool_used + rows > h->cfg.pool_tokens) return SFM_ECAPACITY;
+  Session& s = h->sessions[slot];
+  s.open = true;
+  s.cache_units = cache_units;
+  s.base_row = h->pool_used;
+  s.units = 0;
+  h->pool_used += rows;
+  *session = slot;
+  return SFM_OK;
+}
+
+int sfm_session_reset(sfm_handle* h, int session) {
+  int rc = session_ok(h, session);
+  if (rc) return rc;
+  h->sessions[session].units = 0;
+  return SFM_OK;
+}
+
+int sfm_session_get_info(const sfm_handle* h, int session, sfm_session_info* out) {
+  int rc = session_ok(h, session);
+  if (rc) return rc;
+  if (!out) return SFM_EINVAL;
+  const Session& s = h->sessions[session];
+  out->cache_units = s.cache_units;
+  out->units_appended = s.units;
+  out->valid_tokens = valid_tokens(h, s);
+  out->p0 = s.units * h->cfg.unit_kv_tokens;
+  out->base_row = s.base_row;
+  return SFM_OK;
+}
+
+int sfm_kvcache_append(sfm_handle* h, int session, const void* k, const void* v, int n_tok,
+                       void* stream) {
+  int rc = session_ok(h, session);
+  if (rc) return rc;
+  if (!k || !v || !aligned16(k) || !aligned16(v)) return SFM_EINVAL;
+  const int T = h->cfg.unit_kv_tokens;
+  if (n_tok <= 0 || n_tok % T) return SFM_EINVAL;
+  Session& s = h->sessions[session];
+  long long n_units = n_tok / T;
+  if (!h->cfg.ring && s.units + n_units > s.cache_units) return SFM_ECAPACITY;
+  // With the ring on, only the last cache_units units of a long slice survive.
+  long long skip = n_units > s.cache_units ? n_units - s.cache_units : 0;
+  const long long first = s.units + skip;
+  const size_t row_bytes = (size_t)h->hd * h->es;
+  const char* ks = (const char*)k + skip * T * row_bytes;
+  const char* vs = (const char*)v + skip * T * row_bytes;
+  // the kernel reads rows layer * n_tok + t of the caller's slice; with a skip,
+  // each layer's rows start skip * T rows later inside that layer
+  ProfScope ps(SFM_PROF_APPEND, (cudaStream_t)stream);
+  if (skip) {
+    // copy layer by layer so the per-layer source stride stays n_tok
+    for (int l = 0; l < h->cfg.n_layers; ++l) {
+      rc = launch_kv_append(ks + (size_t)l * n_tok * row_bytes, vs + (size_t)l * n_tok * row_bytes,
+                            h->layer_k(l), h->layer_v(l), 1, h->cfg.pool_tokens, (int)row_bytes,
+                            (int)((n_units - skip) * T), T, s.base_row, first % s.cache_units,
+                            s.cache_units, (cudaStream_t)stream);
+      if (rc) return rc;
+    }
+  } else {
+    rc = launch_kv_append(k, v, h->k_pool, h->v_pool, h->cfg.n_layers, h->cfg.pool_tokens,
+                          (int)row_bytes, n_tok, T, s.base_row, first % s.cache_units,
+                          s.cache_units, (cudaStream_t)stream);
+    if (rc) return rc;
+  }
+  s.units += n_units;
+  return SFM_OK;
+}
+
+int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long long row0,
+                     long long n_rows, void* k_dst, void* v_dst, void* stream) {
+  int rc = session_ok(h, session);
+  if (rc) return rc;
+  const Session& s = h->sessions[session];
+  const long long cap = (long long)s.cache_units * h->cfg.unit_kv_tokens + h->n_tok;
+  if (layer < 0 || layer >= h->cfg.n_layers || row0 < 0 || n_rows < 0 || row0 + n_rows > cap)
+    return SFM_EINVAL;
+  if (n_rows > 0 && (!k_dst || !v_dst || !aligned16(k_dst) || !aligned16(v_dst)))
+    return SFM_EINVAL;
+  return launch_kv_read(h->k_pool, h->v_pool, k_dst, v_dst, layer, h->cfg.pool_tokens,
+                        h->hd * h->es, s.base_row + row0, n_rows, (cudaStream_t)stream);
+}
+
+int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_from, float tau_to,
+                     float* v_out, void* stream) {
+  int rc = session_ok(h, session);
+  if (rc) return rc;
+  if (!h->has_weights || !z || !isfinite(tau_from) || !isfinite(tau_to)) return SFM_EINVAL;
+  const float taus[2] = {tau_from, tau_to};
+  float* zs[1] = {z};
+  float* vs[1] = {v_out};
+  return solve(h, 1, &session, zs, taus, 2, vs, (cudaStream_t)stream);
+}
+
+int sfm_fm_solve(sfm_handle* h, int session, float* z, const float* taus, int n_taus,
+                 void* stream) {
+  int rc = session_ok(h, session);
+  if (rc) return rc;
+  if (!h->has_weights || !z) return SFM_EINVAL;
+  if ((rc = check_taus(taus, n_taus))) return rc;
+  float* zs[1] = {z};
+  return solve(h, 1, &session, zs, taus, n_taus, nullptr, (cudaStream_t)stream);
+}
+
+int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions, float* const* z,
+                         const float* taus, int n_taus, void* stream) {
+  if (!h || !sessions || !z || n_sessions < 1) return SFM_EINVAL;
+  if (!h->has_weights) return SFM_EINVAL;
+  if (n_sessions > h->cfg.max_sessions) return SFM_ECAPACITY;
+  int rc;
+  for (int i = 0; i < n_sessions; ++i) {
+    if ((rc = session_ok(h, sessions[i]))) return rc;
+    if (!z[i]) return SFM_EINVAL;
+    for (int j = 0; j < i; ++j)
+      if (sessions[j] == sessions[i]) return SFM_EINVAL;
+  }
+  if ((rc = check_taus(taus, n_taus))) return rc;
+  return solve(h, n_sessions, sessions, z, taus, n_taus, nullptr, (cudaStream_t)stream);
+}
+
+size_t sfm_attention_workspace_bytes(int n_q, int n_kv, int n_heads, int head_dim, int dtype) {
+  if (dtype != SFM_DTYPE_BF16 || n_q < 1 || n_kv < 1 || n_heads < 1 || head_dim != 128) return 0;
+  const int splits = attention_splits(n_q, 1, n_kv, n_heads);
+  return attention_workspace_bytes(n_q, n_heads, splits);
+}
+
+int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q, int n_kv,
+                  int n_heads, int head_dim, int dtype, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  if (!q || !k || !v || !o || n_q < 1 || n_kv < 1 || n_heads < 1) return SFM_EINVAL;
+  if (dtype != SFM_DTYPE_BF16 && dtype != SFM_DTYPE_FP32) return SFM_EINVAL;
+  if (dtype == SFM_DTYPE_BF16 && head_dim != 128) return SFM_EUNSUPPORTED;
+  if (dtype == SFM_DTYPE_FP32 && (head_dim % 32 || head_dim > 128 || head_dim < 32))
+    return SFM_EUNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SFM_EINVAL;
+  const size_t need = sfm_attention_workspace_bytes(n_q, n_kv, n_heads, head_dim, dtype);
+  if (workspace_bytes < need || (need && (!workspace || !aligned16(workspace)))) return SFM_EINVAL;
+  AttnDesc a{};
+  a.n = 1;
+  a.rows_per = n_q;
+  a.kbase[0] = 0;
+  a.nkeys[0] = n_kv;
+  int splits = 1;
+  float *o_part = nullptr, *lse_part = nullptr;
+  if (dtype == SFM_DTYPE_BF16) {
+    splits = attention_splits(n_q, 1, n_kv, n_heads);
+    if (splits > 1) {
+      o_part = (float*)workspace;
+      lse_part = o_part + (size_t)splits * n_q * n_heads * 128;
+    }
+  }
+  return launch_attention(a, q, k, v, o, n_heads, head_dim, dtype, splits, o_part, lse_part,
+                          (cudaStream_t)stream);
+}
+
+int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream) {
+  if (n < 0 || (n > 0 && (!z || !v || !aligned16(z) || !aligned16(v))) || !isfinite(dtau))
+    return SFM_EINVAL;
+  return launch_euler(z, v, dtau, n, (cudaStream_t)stream);
+}
+
+const char* sfm_strerror(int status) {
+  switch (status) {
+    case SFM_OK: return "ok";
+    case SFM_EINVAL: return "invalid argument";
+    case SFM_ECAPACITY: return "capacity exceeded";
+    case SFM_ESESSION: return "unknown or closed session";
+    case SFM_ECUDA: return "CUDA error";
+    case SFM_ENOMEM: return "device allocation failed";
+    case SFM_EUNSUPPORTED: return "unsupported shape";
+    default: return "unknown status";
+  }
+}
+
+int sfm_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

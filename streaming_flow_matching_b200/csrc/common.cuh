@@ -1,0 +1,81 @@
+// Internal definitions shared by the kernels and the C-ABI of libsfm.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "sfm.h"
+
+namespace sfm {
+
+// Largest batch of sessions one call can carry (kernel parameters hold the
+// per-session table by value, so batched launches stay graph-capturable).
+constexpr int kMaxBatch = 16;
+
+// Per-call description of the sessions in a batch; row r of the activations
+// belongs to session r / n_tok, token r % n_tok.
+struct BatchDesc {
+  int n;                     // sessions in the batch
+  int n_tok;                 // N: tokens of one unit
+  int n_video;               // video tokens (the rest are audio)
+  long long base[kMaxBatch]; // first pool row of each session's region
+  int valid[kMaxBatch];      // S_c: valid cached tokens
+  long long p0[kMaxBatch];   // position of the unit's first token
+};
+
+struct Session {
+  bool open = false;
+  int cache_units = 0;
+  long long base_row = 0;
+  long long units = 0;
+};
+
+int record_cuda(cudaError_t e);  // stores e for sfm_last_cuda_error; returns SFM_ECUDA or SFM_OK
+void count_launch();             // one more kernel launched by this library
+
+// Records a CUDA event pair around the launches in its scope when the
+// profiler is on (sfm_profile_begin); no-op otherwise.
+class ProfScope {
+ public:
+  ProfScope(int kind, cudaStream_t s);
+  ~ProfScope();
+  ProfScope(const ProfScope&) = delete;
+  ProfScope& operator=(const ProfScope&) = delete;
+
+ private:
+  int idx_ = -1;
+  cudaStream_t s_;
+};
+
+// Launch helpers (each returns 0 / SFM_ECUDA after checking cudaGetLastError).
+int launch_kv_append(const void* k, const void* v, void* k_pool, void* v_pool, int n_layers,
+                     long long pool_tokens, int row_bytes, int n_tok, int unit_tokens,
+                     long long base_row, long long first_unit, int cache_units, cudaStream_t s);
+int launch_kv_read(const void* k_pool, const void* v_pool, void* k_dst, void* v_dst, int layer,
+                   long long pool_tokens, int row_bytes, long long row0, long long n_rows,
+                   cudaStream_t s);
+
+int launch_embed(const BatchDesc& b, float* const* z, const void* w_in, const void* e_mod,
+                 float tau, float* x, int d, int c_lat, int dtype, cudaStream_t s);
+int launch_rmsnorm(const float* x, const void* g, void* out, int rows, int d, float eps,
+                   int dtype, cudaStream_t s);
+int launch_rope_table(const BatchDesc& b, float* cos_t, float* sin_t, int head_dim,
+                      double theta, cudaStream_t s);
+int launch_rope_scatter(const BatchDesc& b, const float* qkv, const float* cos_t,
+                        const float* sin_t, void* q_out, void* k_layer, void* v_layer,
+                        int n_heads, int head_dim, int dtype, cudaStream_t s);
+int launch_head_euler(const BatchDesc& b, const float* x, const void* g, const void* w_out,
+                      float* const* z, float* const* v_out, float dtau, int d, int c_lat,
+                      float eps, int dtype, cudaStream_t s);
+int launch_euler(float* z, const float* v, float dtau, long long n, cudaStream_t s);
+
+// GEMM C = A B^T, A [M][K], B [N][K] (both K-contiguous).
+enum Epilogue { EPI_F32 = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_STORE = 3 };
+int launch_gemm(const void* A, const void* B, void* C, int M, int N, int K, int epi, int dtype,
+                cudaStream_t s);
+
+}  // namespace sfm

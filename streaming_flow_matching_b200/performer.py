@@ -1,0 +1,178 @@
+"""Thin Python binding over libsfm for torch tensors: argument marshalling only.
+
+Every computation runs in libsfm's CUDA kernels; this module only turns
+torch tensors into device pointers, passes the current CUDA stream, and turns
+status codes into exceptions.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import torch
+
+from . import _lib as L
+
+_DT = {torch.bfloat16: L.SFM_DTYPE_BF16, torch.float32: L.SFM_DTYPE_FP32}
+
+
+def _stream():
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return C.c_void_p(t.data_ptr()) if t is not None else C.c_void_p(0)
+
+
+def _need(t, dtype, name, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+class Performer:
+    """One libsfm handle: the weights of f_theta, the K/V pool and its sessions."""
+
+    def __init__(self, *, n_layers, d_model, n_heads, head_dim, d_mlp, c_lat, n_video, n_audio,
+                 unit_kv_tokens, pool_tokens, max_sessions=1, dtype=torch.bfloat16, ring=True,
+                 rope_theta=10000.0, rms_eps=1e-6, weights=None):
+        self.dtype = dtype
+        self.cfg = L.sfm_config(n_layers, d_model, n_heads, head_dim, d_mlp, c_lat, n_video,
+                                n_audio, unit_kv_tokens, max_sessions, pool_tokens, _DT[dtype],
+                                int(ring), rope_theta, rms_eps)
+        self.n_tok = n_video + n_audio
+        self.shape = dict(n_layers=n_layers, n_heads=n_heads, head_dim=head_dim, c_lat=c_lat)
+        self._weights = weights           # keeps the borrowed device memory alive
+        self._h = C.c_void_p()
+        wp = None
+        if weights is not None:
+            wp = self._weights_struct(weights)
+        L.check(L.lib.sfm_create(C.byref(self.cfg), C.byref(wp) if wp is not None else None,
+                                 C.byref(self._h)), "sfm_create")
+
+    @classmethod
+    def from_workload(cls, w, weights, pool_tokens=None, max_sessions=1, ring=True):
+        if pool_tokens is None:
+            pool_tokens = max_sessions * (w.cache_units * w.unit_kv_tokens + w.n_tokens)
+        return cls(n_layers=w.n_layers, d_model=w.d_model, n_heads=w.n_heads,
+                   head_dim=w.head_dim, d_mlp=w.d_mlp, c_lat=w.c_lat, n_video=w.n_video,
+                   n_audio=w.n_audio, unit_kv_tokens=w.unit_kv_tokens, pool_tokens=pool_tokens,
+                   max_sessions=max_sessions,
+                   dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32, ring=ring,
+                   rope_theta=w.rope_theta, rms_eps=w.rms_eps, weights=weights)
+
+    def _weights_struct(self, w):
+        n = self.cfg.n_layers
+        for name in ("w_in", "e_mod", "g_final", "w_out"):
+            _need(w[name], self.dtype, name)
+        arrs = {}
+        for name in ("g_attn", "w_qkv", "w_o", "g_mlp", "w_1", "w_2"):
+            ts = [lw[name] for lw in w["layers"]]
+            if len(ts) != n:
+                raise ValueError(f"weights need {n} layers")
+            for t in ts:
+                _need(t, self.dtype, name)
+            arrs[name] = (C.c_void_p * n)(*[t.data_ptr() for t in ts])
+        self._ptr_arrays = arrs
+        return L.sfm_weights(w["w_in"].data_ptr(), w["e_mod"].data_ptr(), w["g_final"].data_ptr(),
+                             w["w_out"].data_ptr(),
+                             *[C.cast(arrs[k], C.POINTER(C.c_void_p))
+                               for k in ("g_attn", "w_qkv", "w_o", "g_mlp", "w_1", "w_2")])
+
+    # -- sessions -------------------------------------------------------------
+    def open_session(self, cache_units):
+        s = C.c_int()
+        L.check(L.lib.sfm_session_open(self._h, cache_units, C.byref(s)), "sfm_session_open")
+        return s.value
+
+    def reset_session(self, session):
+        L.check(L.lib.sfm_session_reset(self._h, session), "sfm_session_reset")
+
+    def session_info(self, session):
+        info = L.sfm_session_info()
+        L.check(L.lib.sfm_session_get_info(self._h, session, C.byref(info)), "sfm_session_get_info")
+        return {f: getattr(info, f) for f, _ in L.sfm_session_info._fields_}
+
+    # -- hot path ---------------------------------------------------------------
+    def kvcache_append(self, session, k, v):
+        _need(k, self.dtype, "k")
+        _need(v, self.dtype, "v", k.shape)
+        n_tok = k.shape[1]
+        L.check(L.lib.sfm_kvcache_append(self._h, session, _ptr(k), _ptr(v), n_tok, _stream()),
+                "sfm_kvcache_append")
+
+    def kvcache_read(self, session, layer, row0, n_rows):
+        shp = (n_rows, self.shape["n_heads"], self.shape["head_dim"])
+        k = torch.empty(shp, dtype=self.dtype, device="cuda")
+        v = torch.empty(shp, dtype=self.dtype, device="cuda")
+        L.check(L.lib.sfm_kvcache_read(self._h, session, layer, row0, n_rows, _ptr(k), _ptr(v),
+                                       _stream()), "sfm_kvcache_read")
+        return k, v
+
+    def denoise_step(self, session, z, tau_from, tau_to, v_out=None):
+        _need(z, torch.float32, "z", (self.n_tok, self.shape["c_lat"]))
+        if v_out is not None:
+            _need(v_out, torch.float32, "v_out", z.shape)
+        L.check(L.lib.sfm_denoise_step(self._h, session, _ptr(z), tau_from, tau_to, _ptr(v_out),
+                                       _stream()), "sfm_denoise_step")
+
+    def fm_solve(self, session, z, taus):
+        _need(z, torch.float32, "z", (self.n_tok, self.shape["c_lat"]))
+        t = (C.c_float * len(taus))(*taus)
+        L.check(L.lib.sfm_fm_solve(self._h, session, _ptr(z), t, len(taus), _stream()),
+                "sfm_fm_solve")
+
+    def fm_solve_batched(self, sessions, zs, taus):
+        for z in zs:
+            _need(z, torch.float32, "z", (self.n_tok, self.shape["c_lat"]))
+        n = len(sessions)
+        s = (C.c_int * n)(*sessions)
+        zp = (C.c_void_p * n)(*[z.data_ptr() for z in zs])
+        t = (C.c_float * len(taus))(*taus)
+        L.check(L.lib.sfm_fm_solve_batched(self._h, n, s, zp, t, len(taus), _stream()),
+                "sfm_fm_solve_batched")
+
+    def close(self):
+        if self._h:
+            L.lib.sfm_destroy(self._h)
+            self._h = C.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def attention(q, k, v, out=None, workspace=None):
+    """O = softmax(Q K^T / sqrt(D)) V per head, every key visible; q [n_q][H][D], k/v [n_kv][H][D]."""
+    dt = _DT[q.dtype]
+    _need(q, q.dtype, "q")
+    _need(k, q.dtype, "k")
+    _need(v, q.dtype, "v", k.shape)
+    n_q, H, D = q.shape
+    n_kv = k.shape[0]
+    if out is None:
+        out = torch.empty_like(q)
+    need = L.lib.sfm_attention_workspace_bytes(n_q, n_kv, H, D, dt)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    L.check(L.lib.sfm_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), n_q, n_kv, H, D, dt,
+                                _ptr(workspace), ws_bytes, _stream()), "sfm_attention")
+    return out
+
+
+def attention_workspace_bytes(n_q, n_kv, n_heads, head_dim, dtype=torch.bfloat16):
+    return L.lib.sfm_attention_workspace_bytes(n_q, n_kv, n_heads, head_dim, _DT[dtype])
+
+
+def euler_update(z, v, dtau):
+    _need(z, torch.float32, "z")
+    _need(v, torch.float32, "v", z.shape)
+    L.check(L.lib.sfm_euler_update(_ptr(z), _ptr(v), dtau, z.numel(), _stream()),
+            "sfm_euler_update")

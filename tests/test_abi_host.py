@@ -1,0 +1,78 @@
+"""The C-ABI library loads, exports every symbol include/sfm.h declares, and
+rejects bad arguments on the host before touching a GPU (no compute calls)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from streaming_flow_matching_b200 import _lib as L
+
+HEADER_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+
+
+def declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(HEADER_DIR, fn)).read()
+            names += re.findall(r"^SFM_API\s+[\w\s\*]+?\b(sfm_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert len(names) >= 15
+    lib = C.CDLL(L.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(L.EXPORTS) <= set(names)
+
+
+def cfg(**kw):
+    base = dict(n_layers=2, d_model=256, n_heads=4, head_dim=64, d_mlp=1024, c_lat=16,
+                n_video=64, n_audio=4, unit_kv_tokens=96, max_sessions=1, pool_tokens=0,
+                dtype=L.SFM_DTYPE_FP32, ring=1, rope_theta=1e4, rms_eps=1e-6)
+    base.update(kw)
+    return L.sfm_config(*[base[f] for f, _ in L.sfm_config._fields_])
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(n_layers=0), L.SFM_EINVAL),
+    (dict(d_model=0), L.SFM_EINVAL),
+    (dict(n_video=0, n_audio=0), L.SFM_EINVAL),
+    (dict(unit_kv_tokens=0), L.SFM_EINVAL),
+    (dict(dtype=7), L.SFM_EINVAL),
+    (dict(rms_eps=-1.0), L.SFM_EINVAL),
+    (dict(max_sessions=17), L.SFM_EUNSUPPORTED),
+    (dict(c_lat=65), L.SFM_EUNSUPPORTED),
+    (dict(dtype=L.SFM_DTYPE_BF16), L.SFM_EUNSUPPORTED),          # bf16 needs D_h = 128
+    (dict(dtype=L.SFM_DTYPE_BF16, head_dim=128, n_heads=2, d_model=192), L.SFM_EUNSUPPORTED),
+    (dict(head_dim=48), L.SFM_EUNSUPPORTED),
+])
+def test_create_rejects_bad_config_on_host(bad, code):
+    h = C.c_void_p()
+    c = cfg(**bad)
+    assert L.lib.sfm_create(C.byref(c), None, C.byref(h)) == code
+    assert not h.value
+
+
+def test_null_arguments_are_rejected():
+    h = C.c_void_p()
+    assert L.lib.sfm_create(None, None, C.byref(h)) == L.SFM_EINVAL
+    assert L.lib.sfm_create(C.byref(cfg()), None, None) == L.SFM_EINVAL
+    assert L.lib.sfm_session_reset(None, 0) == L.SFM_EINVAL
+    assert L.lib.sfm_kvcache_append(None, 0, None, None, 96, None) == L.SFM_EINVAL
+    assert L.lib.sfm_euler_update(None, None, 0.5, 16, None) == L.SFM_EINVAL
+    assert L.lib.sfm_euler_update(None, None, 0.5, 0, None) == L.SFM_OK   # empty is a no-op
+    assert L.lib.sfm_attention(None, None, None, None, 4, 4, 1, 128, 0, None, 0, None) == L.SFM_EINVAL
+    assert L.lib.sfm_attention_workspace_bytes(924, 58524, 24, 128, L.SFM_DTYPE_FP32) == 0
+    assert L.lib.sfm_strerror(L.SFM_ESESSION) == b"unknown or closed session"
+    assert L.lib.sfm_strerror(12345) == b"unknown status"
+
+
+def test_attention_workspace_grows_with_splits():
+    small = L.lib.sfm_attention_workspace_bytes(924, 1024, 24, 128, L.SFM_DTYPE_BF16)
+    big = L.lib.sfm_attention_workspace_bytes(924, 132924, 24, 128, L.SFM_DTYPE_BF16)
+    assert big >= small
+    assert big % 16 == 0

@@ -1,0 +1,128 @@
+"""Micro-benchmarks of single kernels of the hot path, timed with CUDA events.
+
+  python -m streaming_flow_matching_b200.microbench attention --n-kv 16800 [--n-q 924 --heads 24]
+  python -m streaming_flow_matching_b200.microbench append [--layers 28 --units 1]
+  python -m streaming_flow_matching_b200.microbench euler [--n 268435456]
+  python -m streaming_flow_matching_b200.microbench sweep      # attention + append sweep
+
+Inputs are seeded and larger than L2 where the case allows; each timing is
+the median of --reps launches after --warmup launches.  Prints one JSON line
+per case.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import sfm_synth as S  # noqa: E402
+from streaming_flow_matching_b200 import Performer, attention, attention_workspace_bytes, euler_update  # noqa: E402
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def _time(fn, warmup, reps):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def bench_attention(n_q, n_kv, heads, warmup, reps):
+    q, k, v = S.make_qkv(n_q, n_kv, heads, 128, device="cuda")
+    o = torch.empty_like(q)
+    ws_n = attention_workspace_bytes(n_q, n_kv, heads, 128)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda")
+    ms = _time(lambda: attention(q, k, v, o, ws), warmup, reps)
+    flop = 4.0 * n_q * n_kv * heads * 128
+    hbm, bf16, src = _peaks()
+    tf = flop / (ms / 1e3) / 1e12
+    return {"case": "attention", "n_q": n_q, "n_kv": n_kv, "heads": heads, "ms": ms,
+            "tflops": tf, "frac_of_bf16_burst": tf / bf16, "peak_source": src}
+
+
+def bench_append(layers, units, warmup, reps):
+    w = S.V02.replace(n_layers=layers)
+    p = Performer.from_workload(w, None)
+    s = p.open_session(w.cache_units)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2)
+    shape = (layers, units * w.unit_kv_tokens, w.n_heads, w.head_dim)
+    k = torch.randn(*shape, generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn(*shape, generator=g, device="cuda").to(torch.bfloat16)
+    ms = _time(lambda: p.kvcache_append(s, k, v), warmup, reps)
+    nbytes = 2 * 2 * k.numel() * 2
+    hbm, _, src = _peaks()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    p.close()
+    return {"case": "append", "layers": layers, "units": units, "bytes": nbytes, "ms": ms,
+            "gb_s": gbs, "frac_of_hbm": gbs / hbm, "peak_source": src}
+
+
+def bench_euler(n, warmup, reps):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4)
+    z = torch.randn(n, generator=g, device="cuda")
+    v = torch.randn(n, generator=g, device="cuda")
+    ms = _time(lambda: euler_update(z, v, -0.25), warmup, reps)
+    hbm, _, src = _peaks()
+    gbs = 12.0 * n / (ms / 1e3) / 1e9
+    return {"case": "euler", "n": n, "ms": ms, "gb_s": gbs, "frac_of_hbm": gbs / hbm,
+            "peak_source": src}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["attention", "append", "euler", "sweep"])
+    ap.add_argument("--n-q", type=int, default=924)
+    ap.add_argument("--n-kv", type=int, default=57600 + 924)
+    ap.add_argument("--heads", type=int, default=24)
+    ap.add_argument("--layers", type=int, default=28)
+    ap.add_argument("--units", type=int, default=1)
+    ap.add_argument("--n", type=int, default=1 << 28)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--reps", type=int, default=10)
+    a = ap.parse_args()
+    torch.cuda.set_device(0)
+    out = []
+    if a.case == "attention":
+        out.append(bench_attention(a.n_q, a.n_kv, a.heads, a.warmup, a.reps))
+    elif a.case == "append":
+        out.append(bench_append(a.layers, a.units, a.warmup, a.reps))
+    elif a.case == "euler":
+        out.append(bench_euler(a.n, a.warmup, a.reps))
+    else:
+        for n_kv in S.ATTN_SWEEP_TOKENS:
+            out.append(bench_attention(a.n_q, n_kv + a.n_q, a.heads, a.warmup, a.reps))
+        out.append(bench_append(1, 1, a.warmup, a.reps))
+        out.append(bench_append(a.layers, 1, a.warmup, a.reps))
+        out.append(bench_euler(a.n, a.warmup, a.reps))
+    for o in out:
+        print(json.dumps(o), flush=True)
+
+
+if __name__ == "__main__":
+    main()

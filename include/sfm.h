@@ -200,6 +200,30 @@ SFM_API int sfm_attention(const void* q, const void* k, const void* v, void* o, 
                   int n_heads, int head_dim, int dtype, void* workspace,
                   size_t workspace_bytes, void* stream);
 
+/*
+ * sfm_attention without any allocation.  No counterpart in the paper: this
+ * entry point exists for callers that cannot allocate device memory where they
+ * need attention -- a real-time serving loop with a hard per-unit deadline
+ * (cudaMalloc / cudaFree may synchronise the device and stall it), or a host
+ * program whose own allocator owns all device memory.
+ *   - Same arguments and result as sfm_attention, minus the workspace: the
+ *     split-KV partials live in a fixed array of SFM_NOALLOC_SCRATCH_BYTES
+ *     compiled into the library, which every GPU that loads the library holds
+ *     until the process exits.  The call allocates and frees nothing.
+ *   - Returns SFM_ECAPACITY, launching nothing, when the shape needs more
+ *     scratch than that (sfm_attention_workspace_bytes(...) is the need).
+ *   - The first call on each device resolves the array's device address with
+ *     that device current (cudaGetSymbolAddress); make that first call before
+ *     any stream capture.
+ *   - Every call shares the one array per device, and it keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls that overlap on
+ *     the GPU -- on different streams or from different threads -- race on it:
+ *     order them on one stream.
+ */
+#define SFM_NOALLOC_SCRATCH_BYTES (64u << 20)
+SFM_API int sfm_attention_noalloc(const void* q, const void* k, const void* v, void* o, int n_q,
+                                  int n_kv, int n_heads, int head_dim, int dtype, void* stream);
+
 /* Vectorised Euler update z[i] += dtau * v[i], i < n; device fp32. */
 SFM_API int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream);
 

@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(_HERE, "libsfm.so")
 SFM_OK, SFM_EINVAL, SFM_ECAPACITY, SFM_ESESSION, SFM_ECUDA, SFM_ENOMEM, SFM_EUNSUPPORTED = (
     0, -1, -2, -3, -4, -5, -6)
 SFM_DTYPE_BF16, SFM_DTYPE_FP32 = 0, 1
+SFM_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class sfm_config(C.Structure):
@@ -51,7 +52,7 @@ def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"libsfm.so is not built ({LIB_PATH}); build it with "
-            "`python -m streaming_flow_matching_b200.build`")
+            "`python streaming_flow_matching_b200/build.py`")
     L = C.CDLL(LIB_PATH)
     vp, i, ll, f, sz = C.c_void_p, C.c_int, C.c_longlong, C.c_float, C.c_size_t
     sig = {
@@ -67,6 +68,7 @@ def _load():
         "sfm_fm_solve_batched": (i, [vp, i, C.POINTER(i), C.POINTER(vp), C.POINTER(f), i, vp]),
         "sfm_attention_workspace_bytes": (sz, [i, i, i, i, i]),
         "sfm_attention": (i, [vp, vp, vp, vp, i, i, i, i, i, vp, sz, vp]),
+        "sfm_attention_noalloc": (i, [vp, vp, vp, vp, i, i, i, i, i, vp]),
         "sfm_euler_update": (i, [vp, vp, f, ll, vp]),
         "sfm_profile_begin": (i, [i]),
         "sfm_profile_end": (i, [C.POINTER(C.c_double), C.POINTER(ll)]),
@@ -88,7 +90,7 @@ lib = _load()
 EXPORTS = ["sfm_create", "sfm_destroy", "sfm_session_open", "sfm_session_reset",
            "sfm_session_get_info", "sfm_kvcache_append", "sfm_kvcache_read", "sfm_denoise_step",
            "sfm_fm_solve", "sfm_fm_solve_batched", "sfm_attention_workspace_bytes",
-           "sfm_attention", "sfm_euler_update", "sfm_profile_begin", "sfm_profile_end",
+           "sfm_attention", "sfm_attention_noalloc", "sfm_euler_update", "sfm_profile_begin", "sfm_profile_end",
            "sfm_kernel_launch_count", "sfm_strerror", "sfm_last_cuda_error"]
 
 PROF_KINDS = ["append", "attention", "attention_merge", "gemm_qkv", "gemm_o", "gemm_up",

@@ -1,7 +1,7 @@
 """Performer next-unit flow-matching denoise step on B200: Python binding of libsfm.
 
 Importing this package loads libsfm.so (built in-tree by
-``python -m streaming_flow_matching_b200.build``) and fails if it is missing.
+``python streaming_flow_matching_b200/build.py``) and fails if it is missing.
 """
 from . import _lib
 from ._lib import SfmError, lib  # noqa: F401

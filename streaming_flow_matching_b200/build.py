@@ -1,6 +1,7 @@
 """Builds libsfm.so in-tree from csrc/*.cu with nvcc for sm_100a.
 
-Usage: python -m streaming_flow_matching_b200.build [--force]
+Usage: python streaming_flow_matching_b200/build.py [--force] [--ptxas]
+(run as a file: importing the package itself loads the library this builds)
 Objects go to streaming_flow_matching_b200/_build/; the shared library to
 streaming_flow_matching_b200/libsfm.so.  Incremental: a source is recompiled
 when it, or any header under csrc/ or include/, is newer than its object.

@@ -224,6 +224,21 @@ SFM_API int sfm_attention(const void* q, const void* k, const void* v, void* o, 
 SFM_API int sfm_attention_noalloc(const void* q, const void* k, const void* v, void* o, int n_q,
                                   int n_kv, int n_heads, int head_dim, int dtype, void* stream);
 
+/*
+ * One dense projection of f_theta, y = x W^T: x [M][K], w [N][K] (device,
+ * dtype as given), y [M][N].  epilogue: SFM_LINEAR_F32 writes fp32 y;
+ * SFM_LINEAR_OUT writes y in dtype; SFM_LINEAR_GELU writes GELU_tanh(x W^T) in
+ * dtype; SFM_LINEAR_RESID adds x W^T to an fp32 y in place (the residual
+ * stream).  bf16: N a multiple of 128, K of 64 (tcgen05 tensor cores);
+ * fp32: N a multiple of 64, K of 16 (CUDA cores).
+ */
+#define SFM_LINEAR_F32   0
+#define SFM_LINEAR_OUT   1
+#define SFM_LINEAR_GELU  2
+#define SFM_LINEAR_RESID 3
+SFM_API int sfm_linear(const void* x, const void* w, void* y, int M, int N, int K, int epilogue,
+                       int dtype, void* stream);
+
 /* Vectorised Euler update z[i] += dtau * v[i], i < n; device fp32. */
 SFM_API int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream);
 
@@ -253,6 +268,11 @@ SFM_API int sfm_profile_end(double* ms, long long* launches);
 SFM_API unsigned long long sfm_kernel_launch_count(void);
 
 /* ---- errors --------------------------------------------------------------- */
+/* Synchronises the device and reads the handle's device error word: 0 when no
+ * kernel of this handle has reported a problem; 1 when a bounded wait inside a
+ * tensor-core kernel timed out (the kernel then unwound without finishing its
+ * tile, so results of that call are invalid). */
+SFM_API int sfm_check_device_error(const sfm_handle* h, int* code);
 SFM_API const char* sfm_strerror(int status);
 /* The cudaError_t of the last failed CUDA call made by this library on this
  * host thread (0 if none). */

@@ -5,6 +5,7 @@ Importing this package loads libsfm.so (built in-tree by
 """
 from . import _lib
 from ._lib import SfmError, lib  # noqa: F401
-from .performer import Performer, attention, attention_workspace_bytes, euler_update  # noqa: F401
+from .performer import Performer, attention, attention_workspace_bytes, euler_update, linear  # noqa: F401
 
-__all__ = ["Performer", "attention", "attention_workspace_bytes", "euler_update", "SfmError", "lib"]
+__all__ = ["Performer", "attention", "attention_workspace_bytes", "euler_update", "linear", "SfmError",
+           "lib"]

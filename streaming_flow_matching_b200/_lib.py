@@ -15,6 +15,7 @@ SFM_OK, SFM_EINVAL, SFM_ECAPACITY, SFM_ESESSION, SFM_ECUDA, SFM_ENOMEM, SFM_EUNS
     0, -1, -2, -3, -4, -5, -6)
 SFM_DTYPE_BF16, SFM_DTYPE_FP32 = 0, 1
 SFM_NOALLOC_SCRATCH_BYTES = 64 << 20
+SFM_LINEAR_F32, SFM_LINEAR_OUT, SFM_LINEAR_GELU, SFM_LINEAR_RESID = 0, 1, 2, 3
 
 
 class sfm_config(C.Structure):
@@ -69,6 +70,8 @@ def _load():
         "sfm_attention_workspace_bytes": (sz, [i, i, i, i, i]),
         "sfm_attention": (i, [vp, vp, vp, vp, i, i, i, i, i, vp, sz, vp]),
         "sfm_attention_noalloc": (i, [vp, vp, vp, vp, i, i, i, i, i, vp]),
+        "sfm_linear": (i, [vp, vp, vp, i, i, i, i, i, vp]),
+        "sfm_check_device_error": (i, [vp, C.POINTER(i)]),
         "sfm_euler_update": (i, [vp, vp, f, ll, vp]),
         "sfm_profile_begin": (i, [i]),
         "sfm_profile_end": (i, [C.POINTER(C.c_double), C.POINTER(ll)]),
@@ -90,8 +93,9 @@ lib = _load()
 EXPORTS = ["sfm_create", "sfm_destroy", "sfm_session_open", "sfm_session_reset",
            "sfm_session_get_info", "sfm_kvcache_append", "sfm_kvcache_read", "sfm_denoise_step",
            "sfm_fm_solve", "sfm_fm_solve_batched", "sfm_attention_workspace_bytes",
-           "sfm_attention", "sfm_attention_noalloc", "sfm_euler_update", "sfm_profile_begin", "sfm_profile_end",
-           "sfm_kernel_launch_count", "sfm_strerror", "sfm_last_cuda_error"]
+           "sfm_attention", "sfm_attention_noalloc", "sfm_linear", "sfm_euler_update", "sfm_profile_begin", "sfm_profile_end",
+           "sfm_kernel_launch_count", "sfm_check_device_error", "sfm_strerror",
+           "sfm_last_cuda_error"]
 
 PROF_KINDS = ["append", "attention", "attention_merge", "gemm_qkv", "gemm_o", "gemm_up",
               "gemm_down", "rowops", "head_euler"]

@@ -8,6 +8,8 @@
 
 #include "attn.cuh"
 #include "common.cuh"
+#include "gemm_tc.cuh"
+#include "sm100.cuh"
 
 using namespace sfm;
 
@@ -45,6 +47,12 @@ struct sfm_handle {
   float* sin_t = nullptr;
   float* o_part = nullptr;   // [kMaxSplits][M][H][D]
   float* lse_part = nullptr; // [kMaxSplits][M][H]
+  int* d_err = nullptr;      // device error word (bounded waits that timed out)
+  int sms = 148;
+  // TMA tensor maps (bf16 mode): activations over max_sessions * N rows, weights per layer
+  CUtensorMap map_xn{}, map_ao{}, map_hmlp{};
+  CUtensorMap map_q{}, map_kpool{}, map_vpool{};  // attention operands
+  std::vector<CUtensorMap> map_wqkv, map_wo, map_w1, map_w2;
   std::vector<void*> owned;
 
   void* layer_k(int l) const { return (char*)k_pool + (size_t)l * cfg.pool_tokens * hd * es; }
@@ -64,6 +72,7 @@ int validate_config(const sfm_config* c) {
   if (c->dtype != SFM_DTYPE_BF16 && c->dtype != SFM_DTYPE_FP32) return SFM_EINVAL;
   if (!(c->rms_eps >= 0.0) || !(c->rope_theta > 0.0)) return SFM_EINVAL;
   if (c->max_sessions > kMaxBatch) return SFM_EUNSUPPORTED;
+  if ((long long)c->n_layers * c->pool_tokens >= (1LL << 31)) return SFM_EUNSUPPORTED;
   if (c->c_lat > 64 || c->d_model % 2) return SFM_EUNSUPPORTED;
   const int hd = c->n_heads * c->head_dim;
   if (c->dtype == SFM_DTYPE_BF16) {
@@ -127,6 +136,41 @@ AttnDesc attn_desc(const BatchDesc& b) {
   return a;
 }
 
+int make_a_map(CUtensorMap* m, const void* p, long long rows, int k) {
+  const uint64_t dims[2] = {(uint64_t)k, (uint64_t)rows};
+  const uint64_t strides[1] = {(uint64_t)k * 2};
+  const uint32_t box[2] = {64, 128};
+  return make_tmap_bf16(m, p, 2, dims, strides, box);
+}
+
+int make_b_map(CUtensorMap* m, const void* p, int n, int k, int block_n) {
+  const uint64_t dims[2] = {(uint64_t)k, (uint64_t)n};
+  const uint64_t strides[1] = {(uint64_t)k * 2};
+  const uint32_t box[2] = {64, (uint32_t)block_n};
+  return make_tmap_bf16(m, p, 2, dims, strides, box);
+}
+
+// rows of [rows][H][128] bf16 (queries, or keys / values), box 128 rows x 64 dims of one head
+int make_rows_map(CUtensorMap* m, const void* p, long long rows, int heads) {
+  const uint64_t dims[3] = {128, (uint64_t)heads, (uint64_t)rows};
+  const uint64_t strides[2] = {256, (uint64_t)heads * 256};
+  const uint32_t box[3] = {64, 1, 128};
+  return make_tmap_bf16(m, p, 3, dims, strides, box);
+}
+
+GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err) {
+  GemmArgs g{};
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.epi = epi;
+  g.C = C;
+  g.ldc = ldc;
+  g.err = err;
+  g.hd = 0;
+  return g;
+}
+
 // One Euler step of f_theta for the sessions in b (RoPE table already filled).
 int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from, float tau_to,
              float* const* v_out, cudaStream_t s) {
@@ -135,8 +179,10 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
   const int d = c.d_model, hd = h->hd, F = c.d_mlp, dt = c.dtype;
   const float eps = (float)c.rms_eps;
   int rc;
-#define SFM_TRY(call) \
-  if ((rc = (call)) != SFM_OK) return rc;
+#define SFM_TRY(call)                \
+  do {                               \
+    if ((rc = (call)) != SFM_OK) return rc; \
+  } while (0)
   {
     ProfScope ps(SFM_PROF_ROWOPS, s);
     SFM_TRY(launch_embed(b, z, h->w_in, h->e_mod, tau_from, h->x, d, c.c_lat, dt, s));
@@ -144,26 +190,50 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
   const AttnDesc ad = attn_desc(b);
   long long max_keys = 0;
   for (int i = 0; i < b.n; ++i) max_keys = ad.nkeys[i] > max_keys ? ad.nkeys[i] : max_keys;
-  const int splits = dt == SFM_DTYPE_BF16 ? attention_splits(b.n_tok, b.n, max_keys, c.n_heads) : 1;
+  const bool tc = dt == SFM_DTYPE_BF16;
+  const int splits = tc ? attention_tc_splits(b.n_tok, b.n, max_keys, c.n_heads, h->sms) : 1;
   for (int l = 0; l < c.n_layers; ++l) {
     {
       ProfScope ps(SFM_PROF_ROWOPS, s);
       SFM_TRY(launch_rmsnorm(h->x, h->g_attn[l], h->xn, M, d, eps, dt, s));
     }
-    {
+    if (tc) {
+      // QKV projection with RoPE and the cache-tail scatter fused in the epilogue
       ProfScope ps(SFM_PROF_GEMM_QKV, s);
-      SFM_TRY(launch_gemm(h->xn, h->w_qkv[l], h->qkv32, M, 3 * hd, d, EPI_F32, dt, s));
-    }
-    {
+      GemmArgs g = gemm_args(M, 3 * hd, d, EPI_QKV, nullptr, 0, h->d_err);
+      g.cos_t = h->cos_t;
+      g.sin_t = h->sin_t;
+      g.q_out = (__nv_bfloat16*)h->q;
+      g.k_layer = (__nv_bfloat16*)h->layer_k(l);
+      g.v_layer = (__nv_bfloat16*)h->layer_v(l);
+      g.hd = hd;
+      g.b = b;
+      SFM_TRY(launch_gemm_tc(h->map_xn, h->map_wqkv[l], g, h->sms, s));
+    } else {
+      {
+        ProfScope ps(SFM_PROF_GEMM_QKV, s);
+        SFM_TRY(launch_gemm(h->xn, h->w_qkv[l], h->qkv32, M, 3 * hd, d, EPI_F32, dt, s));
+      }
       ProfScope ps(SFM_PROF_ROWOPS, s);
       SFM_TRY(launch_rope_scatter(b, h->qkv32, h->cos_t, h->sin_t, h->q, h->layer_k(l),
                                   h->layer_v(l), c.n_heads, c.head_dim, dt, s));
     }
-    SFM_TRY(launch_attention(ad, h->q, h->layer_k(l), h->layer_v(l), h->ao, c.n_heads,
-                             c.head_dim, dt, splits, h->o_part, h->lse_part, s));
+    if (tc) {
+      SFM_TRY(launch_attention_tc(h->map_q, h->map_kpool, h->map_vpool, ad,
+                                  (int)((long long)l * c.pool_tokens), c.n_heads, splits, h->ao,
+                                  h->o_part, h->lse_part, h->d_err, s));
+    } else {
+      SFM_TRY(launch_attention(ad, h->q, h->layer_k(l), h->layer_v(l), h->ao, c.n_heads,
+                               c.head_dim, dt, splits, h->o_part, h->lse_part, s));
+    }
     {
       ProfScope ps(SFM_PROF_GEMM_O, s);
-      SFM_TRY(launch_gemm(h->ao, h->w_o[l], h->x, M, d, hd, EPI_RESID, dt, s));
+      if (tc) {
+        SFM_TRY(launch_gemm_tc(h->map_ao, h->map_wo[l],
+                               gemm_args(M, d, hd, EPI_RESID, h->x, d, h->d_err), h->sms, s));
+      } else {
+        SFM_TRY(launch_gemm(h->ao, h->w_o[l], h->x, M, d, hd, EPI_RESID, dt, s));
+      }
     }
     {
       ProfScope ps(SFM_PROF_ROWOPS, s);
@@ -171,11 +241,21 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
     }
     {
       ProfScope ps(SFM_PROF_GEMM_UP, s);
-      SFM_TRY(launch_gemm(h->xn, h->w_1[l], h->hmlp, M, F, d, EPI_GELU, dt, s));
+      if (tc) {
+        SFM_TRY(launch_gemm_tc(h->map_xn, h->map_w1[l],
+                               gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->d_err), h->sms, s));
+      } else {
+        SFM_TRY(launch_gemm(h->xn, h->w_1[l], h->hmlp, M, F, d, EPI_GELU, dt, s));
+      }
     }
     {
       ProfScope ps(SFM_PROF_GEMM_DOWN, s);
-      SFM_TRY(launch_gemm(h->hmlp, h->w_2[l], h->x, M, d, F, EPI_RESID, dt, s));
+      if (tc) {
+        SFM_TRY(launch_gemm_tc(h->map_hmlp, h->map_w2[l],
+                               gemm_args(M, d, F, EPI_RESID, h->x, d, h->d_err), h->sms, s));
+      } else {
+        SFM_TRY(launch_gemm(h->hmlp, h->w_2[l], h->x, M, d, F, EPI_RESID, dt, s));
+      }
     }
   }
   {
@@ -273,6 +353,47 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     if (!rc && cfg->dtype == SFM_DTYPE_BF16) {
       rc = dalloc(h, &h->o_part, (size_t)kMaxSplits * M * hd * 4);
       if (!rc) rc = dalloc(h, &h->lse_part, (size_t)kMaxSplits * M * cfg->n_heads * 4);
+    }
+  }
+  if (!rc) rc = dalloc(h, &h->d_err, sizeof(int));
+  // Zero everything once: rows a tile reads past a session's valid range must hold
+  // finite values, never uninitialised bit patterns.
+  if (!rc) {
+    if (cudaMemset(h->k_pool, 0, pool_bytes) != cudaSuccess ||
+        cudaMemset(h->v_pool, 0, pool_bytes) != cudaSuccess ||
+        cudaMemset(h->d_err, 0, sizeof(int)) != cudaSuccess)
+      rc = record_cuda(cudaGetLastError());
+    if (!rc && h->has_weights &&
+        (cudaMemset(h->xn, 0, M * d * es) != cudaSuccess ||
+         cudaMemset(h->q, 0, M * hd * es) != cudaSuccess ||
+         cudaMemset(h->ao, 0, M * hd * es) != cudaSuccess ||
+         cudaMemset(h->hmlp, 0, M * F * es) != cudaSuccess))
+      rc = record_cuda(cudaGetLastError());
+  }
+  if (!rc) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  if (!rc && h->has_weights && cfg->dtype == SFM_DTYPE_BF16) {
+    const int L_ = cfg->n_layers, d_ = cfg->d_model, hd_ = h->hd, F_ = cfg->d_mlp;
+    rc = make_a_map(&h->map_xn, h->xn, (long long)M, d_);
+    if (!rc) rc = make_rows_map(&h->map_q, h->q, (long long)M, cfg->n_heads);
+    if (!rc && cfg->pool_tokens > 0)
+      rc = make_rows_map(&h->map_kpool, h->k_pool, (long long)L_ * cfg->pool_tokens, cfg->n_heads);
+    if (!rc && cfg->pool_tokens > 0)
+      rc = make_rows_map(&h->map_vpool, h->v_pool, (long long)L_ * cfg->pool_tokens, cfg->n_heads);
+    if (!rc) rc = make_a_map(&h->map_ao, h->ao, (long long)M, hd_);
+    if (!rc) rc = make_a_map(&h->map_hmlp, h->hmlp, (long long)M, F_);
+    h->map_wqkv.resize(L_);
+    h->map_wo.resize(L_);
+    h->map_w1.resize(L_);
+    h->map_w2.resize(L_);
+    for (int l = 0; l < L_ && !rc; ++l) {
+      rc = make_b_map(&h->map_wqkv[l], h->w_qkv[l], 3 * hd_, d_, gemm_tc_block_n(3 * hd_, hd_, EPI_QKV));
+      if (!rc) rc = make_b_map(&h->map_wo[l], h->w_o[l], d_, hd_, gemm_tc_block_n(d_, 0, EPI_RESID));
+      if (!rc) rc = make_b_map(&h->map_w1[l], h->w_1[l], F_, d_, gemm_tc_block_n(F_, 0, EPI_GELU));
+      if (!rc) rc = make_b_map(&h->map_w2[l], h->w_2[l], d_, F_, gemm_tc_block_n(d_, 0, EPI_RESID));
     }
   }
   if (rc) {
@@ -420,9 +541,13 @@ int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions, flo
   return solve(h, n_sessions, sessions, z, taus, n_taus, nullptr, (cudaStream_t)stream);
 }
 
+// The standalone call chooses its split count for a 148-SM B200 whatever the
+// device, so the workspace it needs is a pure function of the shape.
+constexpr int kStandaloneSms = 148;
+
 size_t sfm_attention_workspace_bytes(int n_q, int n_kv, int n_heads, int head_dim, int dtype) {
   if (dtype != SFM_DTYPE_BF16 || n_q < 1 || n_kv < 1 || n_heads < 1 || head_dim != 128) return 0;
-  const int splits = attention_splits(n_q, 1, n_kv, n_heads);
+  const int splits = attention_tc_splits(n_q, 1, n_kv, n_heads, kStandaloneSms);
   return attention_workspace_bytes(n_q, n_heads, splits);
 }
 
@@ -442,23 +567,66 @@ int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q,
   a.rows_per = n_q;
   a.kbase[0] = 0;
   a.nkeys[0] = n_kv;
-  int splits = 1;
+  if (dtype == SFM_DTYPE_FP32)
+    return launch_attention(a, q, k, v, o, n_heads, head_dim, dtype, 1, nullptr, nullptr,
+                            (cudaStream_t)stream);
+  const int splits = attention_tc_splits(n_q, 1, n_kv, n_heads, kStandaloneSms);
   float *o_part = nullptr, *lse_part = nullptr;
-  if (dtype == SFM_DTYPE_BF16) {
-    splits = attention_splits(n_q, 1, n_kv, n_heads);
-    if (splits > 1) {
-      o_part = (float*)workspace;
-      lse_part = o_part + (size_t)splits * n_q * n_heads * 128;
-    }
+  if (splits > 1) {
+    o_part = (float*)workspace;
+    lse_part = o_part + (size_t)splits * n_q * n_heads * 128;
   }
-  return launch_attention(a, q, k, v, o, n_heads, head_dim, dtype, splits, o_part, lse_part,
-                          (cudaStream_t)stream);
+  CUtensorMap mq, mk, mv;
+  int rc = make_rows_map(&mq, q, n_q, n_heads);
+  if (!rc) rc = make_rows_map(&mk, k, n_kv, n_heads);
+  if (!rc) rc = make_rows_map(&mv, v, n_kv, n_heads);
+  if (rc) return rc;
+  return launch_attention_tc(mq, mk, mv, a, 0, n_heads, splits, o, o_part, lse_part, nullptr,
+                             (cudaStream_t)stream);
 }
 
 int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream) {
   if (n < 0 || (n > 0 && (!z || !v || !aligned16(z) || !aligned16(v))) || !isfinite(dtau))
     return SFM_EINVAL;
   return launch_euler(z, v, dtau, n, (cudaStream_t)stream);
+}
+
+int sfm_check_device_error(const sfm_handle* h, int* code) {
+  if (!h || !code) return SFM_EINVAL;
+  int v = 0;
+  const cudaError_t e = cudaMemcpy(&v, h->d_err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return record_cuda(e);
+  *code = v;
+  return SFM_OK;
+}
+
+int sfm_linear(const void* x, const void* w, void* y, int M, int N, int K, int epilogue,
+               int dtype, void* stream) {
+  if (!x || !w || !y || M < 1 || N < 1 || K < 1) return SFM_EINVAL;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return SFM_EINVAL;
+  int epi;
+  switch (epilogue) {
+    case SFM_LINEAR_F32: epi = EPI_F32; break;
+    case SFM_LINEAR_OUT: epi = EPI_STORE; break;
+    case SFM_LINEAR_GELU: epi = EPI_GELU; break;
+    case SFM_LINEAR_RESID: epi = EPI_RESID; break;
+    default: return SFM_EINVAL;
+  }
+  if (dtype == SFM_DTYPE_FP32) {
+    if (N % 64 || K % 16) return SFM_EUNSUPPORTED;
+    return launch_gemm(x, w, y, M, N, K, epi, dtype, (cudaStream_t)stream);
+  }
+  if (dtype != SFM_DTYPE_BF16) return SFM_EINVAL;
+  if (N % 128 || K % 64) return SFM_EUNSUPPORTED;
+  const int bn = gemm_tc_block_n(N, 0, epi);
+  CUtensorMap ma, mb;
+  int rc = make_a_map(&ma, x, M, K);
+  if (!rc) rc = make_b_map(&mb, w, N, K, bn);
+  if (rc) return rc;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return launch_gemm_tc(ma, mb, gemm_args(M, N, K, epi, y, N, nullptr), sms, (cudaStream_t)stream);
 }
 
 const char* sfm_strerror(int status) {

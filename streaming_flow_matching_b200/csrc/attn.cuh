@@ -1,5 +1,7 @@
 // Attention launch interface shared by the C-ABI and the attention kernels.
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace sfm {
@@ -20,5 +22,18 @@ size_t attention_workspace_bytes(long long rows, int n_heads, int n_splits);
 int launch_attention(const AttnDesc& a, const void* q, const void* k, const void* v, void* o,
                      int n_heads, int head_dim, int dtype, int n_splits, float* o_part,
                      float* lse_part, cudaStream_t s);
+
+int launch_attention_merge(const float* o_part, const float* lse_part, void* o,
+                           long long total_rows, int n_heads, int n_splits, cudaStream_t s);
+
+// tcgen05 attention (bf16, D = 128).  Split count for a batch; the SM count is
+// an input so the choice is reproducible (the standalone call assumes 148).
+int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads,
+                        int sms);
+// mq: map over the query rows [rows][H][128]; mk, mv: maps over the key rows, of
+// which this call uses rows kv_row0 + kbase[s] + [0, nkeys[s]).
+int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const AttnDesc& a, int kv_row0, int n_heads, int n_splits, void* o,
+                        float* o_part, float* lse_part, int* err, cudaStream_t s);
 
 }  // namespace sfm

@@ -358,6 +358,11 @@ int launch_attention(const AttnDesc& a, const void* q, const void* k, const void
   }
   if (rc || n_splits == 1) return rc;
   ProfScope ps(SFM_PROF_ATTN_MERGE, s);
+  return launch_attention_merge(o_part, lse_part, o, total_rows, n_heads, n_splits, s);
+}
+
+int launch_attention_merge(const float* o_part, const float* lse_part, void* o,
+                           long long total_rows, int n_heads, int n_splits, cudaStream_t s) {
   const long long warps = total_rows * n_heads;
   attn_merge_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
       o_part, lse_part, (__nv_bfloat16*)o, total_rows, n_heads, n_splits);

@@ -1,0 +1,430 @@
+// Attention of the current unit on the 5th-generation tensor cores (tcgen05).
+//
+// The performer form of block-causal attention ("Wan-Streamer" v0.1 blog,
+// §3.3): every query of the current unit sees every valid cached key and every
+// key of the current unit, so O = softmax(Q K^T / sqrt(D)) V over one key
+// range per session, D = 128.
+//
+// One CTA = one (session, head, 128-query tile, key split); 192 threads:
+//   warp 0      TMA producer: Q tile once; K tiles (128 keys x 128 dims) in a
+//               3-stage ring, V tiles in a 2-stage ring (128-byte swizzle)
+//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma:
+//                 S_j = Q K_j^T      (M=128, N=128 keys, K=128 dims) into one of
+//                                    two TMEM S buffers, issued two tiles ahead
+//                 O  += P_j V_j      (M=128, N=128 dims, K=128 keys; V as an
+//                                    MN-major operand) into the TMEM O buffer
+//   warps 2-5   softmax, thread = query row: tcgen05.ld of its S row, online
+//               softmax in the exp2 domain, P (bf16) written to shared memory in
+//               the swizzled K-major layout, O rescaled in TMEM only when the
+//               running max grows by more than 2^8 (otherwise the stale max is
+//               kept; P <= 2^8 stays exact in fp32 sums), final O / l written
+//               as bf16 (one split) or as fp32 partials + log2-sum-exp (several).
+// The last, partial key tile is masked in S, and its V rows past the key range
+// are zeroed in shared memory before P V, so rows outside the range never
+// contribute (whatever they hold).
+#include <math.h>
+
+#include "attn.cuh"
+#include "sm100.cuh"
+
+namespace sfm {
+
+using namespace sm100;
+
+namespace atc {
+
+constexpr int BQ = 128, BKV = 128, D = 128;
+constexpr int THREADS = 192;
+constexpr int KST = 3, VST = 2;
+constexpr int HALF = 128 * 64 * 2;        // one [128 rows][64 cols] bf16 swizzle tile: 16 KB
+constexpr int TILE = 2 * HALF;            // [128][128] bf16: 32 KB
+constexpr int OFF_Q = 0;
+constexpr int OFF_P = OFF_Q + TILE;
+constexpr int OFF_K = OFF_P + TILE;
+constexpr int OFF_V = OFF_K + KST * TILE;
+constexpr int OFF_BAR = OFF_V + VST * TILE;      // 229376
+constexpr int SMEM = OFF_BAR + 256 + 1024;
+constexpr uint32_t TMEM_COLS = 512;               // S0 | S1 | O
+constexpr uint32_t COL_O = 256;
+constexpr float kRescaleLog2 = 8.0f;
+
+struct Args {
+  AttnDesc a;
+  int H;
+  int n_splits;
+  int qtiles;
+  float scale_log2;
+  long long total_rows;
+  int kv_row0;                 // row offset of this layer inside the K/V tensor maps
+  __nv_bfloat16* o;            // [total_rows][H][D] (one split)
+  float* o_part;               // [n_splits][total_rows][H][D]
+  float* lse_part;             // [n_splits][total_rows][H]
+  int* err;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                   const __grid_constant__ CUtensorMap map_v, const __grid_constant__ Args args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + VST;
+  uint64_t* s_full = v_empty + VST;   // [2]
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 1;
+  uint64_t* drain = o_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sess = blockIdx.x / args.qtiles;
+  const int qt = blockIdx.x - sess * args.qtiles;
+  const int h = blockIdx.y, split = blockIdx.z;
+  const long long row0 = (long long)sess * args.a.rows_per + qt * BQ;
+  const int q_rows = min(BQ, args.a.rows_per - qt * BQ);
+  const int nkeys = args.a.nkeys[sess];
+  const long long kbase = args.a.kbase[sess];
+  const int ntiles = (nkeys + BKV - 1) / BKV;
+  const int tps = (ntiles + args.n_splits - 1) / args.n_splits;
+  const int t0 = min(ntiles, split * tps);
+  const int t1 = min(ntiles, t0 + tps);
+  const int T = t1 - t0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < KST; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < VST; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&map_q);
+    tma_prefetch(&map_k);
+    tma_prefetch(&map_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && T > 0) {
+      // ---------------- TMA producer ----------------
+      int kp[KST], vp[VST];               // parity of the last load into each stage
+      for (int i = 0; i < KST; ++i) kp[i] = -1;
+      for (int i = 0; i < VST; ++i) vp[i] = -1;
+      bool ok = true;
+      mbar_arrive_expect_tx(q_full, TILE);
+      tma_load_3d(base + OFF_Q, &map_q, q_full, 0, h, (int)row0);
+      tma_load_3d(base + OFF_Q + HALF, &map_q, q_full, 64, h, (int)row0);
+      auto load_k = [&](int i) -> bool {   // i: tile index relative to t0
+        const int s = i % KST;
+        const uint32_t par = (uint32_t)((i / KST) & 1);
+        if (!mbar_wait(&k_empty[s], par ^ 1u, abort, args.err, 0x201)) return false;
+        const int krow = args.kv_row0 + (int)(kbase + (long long)(t0 + i) * BKV);
+        mbar_arrive_expect_tx(&k_full[s], TILE);
+        tma_load_3d(base + OFF_K + s * TILE, &map_k, &k_full[s], 0, h, krow);
+        tma_load_3d(base + OFF_K + s * TILE + HALF, &map_k, &k_full[s], 64, h, krow);
+        kp[s] = (int)par;
+        return true;
+      };
+      auto load_v = [&](int i) -> bool {
+        const int s = i % VST;
+        const uint32_t par = (uint32_t)((i / VST) & 1);
+        if (!mbar_wait(&v_empty[s], par ^ 1u, abort, args.err, 0x202)) return false;
+        const int krow = args.kv_row0 + (int)(kbase + (long long)(t0 + i) * BKV);
+        mbar_arrive_expect_tx(&v_full[s], TILE);
+        tma_load_3d(base + OFF_V + s * TILE, &map_v, &v_full[s], 0, h, krow);
+        tma_load_3d(base + OFF_V + s * TILE + HALF, &map_v, &v_full[s], 64, h, krow);
+        vp[s] = (int)par;
+        return true;
+      };
+      // order of need by the MMA issuer: S_0, S_1, then per j: PV_j, S_{j+2}
+      if (ok && T > 0) ok = load_k(0);
+      if (ok && T > 1) ok = load_k(1);
+      for (int j = 0; j < T && ok; ++j) {
+        ok = load_v(j);
+        if (ok && j + 2 < T) ok = load_k(j + 2);
+      }
+      if (!ok) {   // unwinding: let issued loads land before the CTA exits
+        mbar_drain(q_full, 0);
+        for (int i = 0; i < KST; ++i)
+          if (kp[i] >= 0) mbar_drain(&k_full[i], (uint32_t)kp[i]);
+        for (int i = 0; i < VST; ++i)
+          if (vp[i] >= 0) mbar_drain(&v_full[i], (uint32_t)vp[i]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && T > 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc_s = idesc_bf16(BQ, BKV, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(BQ, D, false, true);
+      bool ok = mbar_wait(q_full, 0, abort, args.err, 0x203), issued = false;
+      auto issue_s = [&](int i) -> bool {
+        const int s = i % KST;
+        if (!mbar_wait(&k_full[s], (uint32_t)((i / KST) & 1), abort, args.err, 0x204)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)((i & 1) * 128);
+        const uint32_t qa = base + OFF_Q, ka = base + OFF_K + s * TILE;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t sub = (uint32_t)(kk >> 2) * HALF;
+          const uint64_t da = sw128_desc(qa + sub, 16, 1024) + (uint64_t)(2 * (kk & 3));
+          const uint64_t db = sw128_desc(ka + sub, 16, 1024) + (uint64_t)(2 * (kk & 3));
+          umma_bf16(d, da, db, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        issued = true;
+        umma_commit(&k_empty[s]);
+        umma_commit(&s_full[i & 1]);
+        return true;
+      };
+      if (ok && T > 0) ok = issue_s(0);
+      if (ok && T > 1) ok = issue_s(1);
+      for (int j = 0; j < T && ok; ++j) {
+        const int vs = j % VST;
+        if (!mbar_wait(p_full, (uint32_t)(j & 1), abort, args.err, 0x205) ||
+            !mbar_wait(&v_full[vs], (uint32_t)((j / VST) & 1), abort, args.err, 0x206)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t pa = base + OFF_P, va = base + OFF_V + vs * TILE;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t da = sw128_desc(pa + (uint32_t)(kk >> 2) * HALF, 16, 1024) +
+                              (uint64_t)(2 * (kk & 3));
+          // V as MN-major B: 64-dim halves HALF bytes apart, 16 keys = 2048 B per K step
+          const uint64_t db = sw128_desc(va + (uint32_t)kk * 2048u, HALF, 1024);
+          umma_bf16(tmem + COL_O, da, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&v_empty[vs]);
+        umma_commit(o_done);
+        if (j + 2 < T) ok = issue_s(j + 2);
+      }
+      if (!ok && issued) {
+        umma_commit(drain);
+        mbar_drain(drain, 0);
+      }
+    }
+  } else {
+    // ---------------- softmax + output (warps 2..5, thread = query row) ----------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                    // row inside the tile
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    uint8_t* prow = smem + OFF_P + r * 128;
+    for (int j = 0; j < T && ok; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (uint32_t)((j >> 1) & 1), abort, args.err, 0x207))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[128];
+      {
+        uint32_t u[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(tmem + lane_base + (uint32_t)((j & 1) * 128 + c * 32), u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(u[i]);
+        }
+      }
+      const int kvalid = nkeys - (t0 + j) * BKV;         // > 0
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        float x = s[i] * args.scale_log2;
+        if (i >= kvalid) x = -INFINITY;
+        s[i] = x;
+        mx = fmaxf(mx, x);
+      }
+      if (j > 0) {
+        // PV_{j-1} must be complete before O is rescaled or P is overwritten
+        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((j - 1) & 1), abort, args.err, 0x208))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      // tcgen05.ld/st are warp-collective: the rescale decision is taken per warp
+      // (any row needing it rescales the whole warp; a row whose max did not grow
+      // gets alpha = 1).
+      if (j == 0) {
+        m = mx;
+      } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+        const float m_new = fmaxf(m, mx);
+        const float alpha = exp2f(m - m_new);
+        l *= alpha;
+        m = m_new;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_base + COL_O + c * 32, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+          tmem_st32(tmem + lane_base + COL_O + c * 32, u);
+        }
+        tmem_st_wait();
+      }
+      // P = exp2(x - m) as bf16 into the swizzled K-major P tile (two 64-key halves)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          p[e] = exp2f(s[c * 8 + e] - m);
+          l += p[e];
+        }
+        uint4 w;
+        w.x = pack_bf16x2(p[0], p[1]);
+        w.y = pack_bf16x2(p[2], p[3]);
+        w.z = pack_bf16x2(p[4], p[5]);
+        w.w = pack_bf16x2(p[6], p[7]);
+        const int half = c >> 3, chunk = c & 7;
+        *reinterpret_cast<uint4*>(prow + half * HALF + ((chunk ^ (r & 7)) << 4)) = w;
+      }
+      if (kvalid < BKV) {
+        // zero the V rows of the partial tile past the key range once the tile has landed
+        const int vs = j % VST;
+        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[vs], (uint32_t)((j / VST) & 1), abort, args.err, 0x209))) {
+          ok = false;
+          break;
+        }
+      }
+      if (kvalid < BKV && r >= kvalid) {
+        const int vs = j % VST;
+        uint4* v0 = reinterpret_cast<uint4*>(smem + OFF_V + vs * TILE + r * 128);
+        uint4* v1 = reinterpret_cast<uint4*>(smem + OFF_V + vs * TILE + HALF + r * 128);
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          v0[q] = z;
+          v1[q] = z;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // ---- output ----
+    if (ok && T > 0) {
+      if (!__all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((T - 1) & 1), abort, args.err, 0x20A))) ok = false;
+      tc_fence_after();
+    }
+    const long long grow = row0 + r;
+    const long long ld = (long long)args.H * D;
+    const bool have = ok && T > 0 && l > 0.f;
+    const float inv = have ? 1.f / l : 0.f;
+    for (int c = 0; c < 4; ++c) {
+      uint32_t u[32];
+      if (T > 0) {
+        tmem_ld32(tmem + lane_base + COL_O + c * 32, u);
+        tmem_ld_wait();
+      }
+      if (r >= q_rows) continue;
+      float o[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = have ? __uint_as_float(u[i]) * inv : 0.f;
+      if (args.n_splits == 1) {
+        uint4* d = reinterpret_cast<uint4*>(args.o + grow * ld + h * D + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          d[q] = make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
+                            pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
+      } else {
+        float4* d = reinterpret_cast<float4*>(args.o_part + ((long long)split * args.total_rows + grow) * ld +
+                                              h * D + c * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) d[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      }
+    }
+    if (r < q_rows && args.n_splits > 1)
+      args.lse_part[((long long)split * args.total_rows + grow) * args.H + h] =
+          have ? m + log2f(l) : -INFINITY;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace atc
+
+int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads,
+                        int sms) {
+  const long long ctas = (long long)n_sessions * ((rows_per_session + atc::BQ - 1) / atc::BQ) * n_heads;
+  const long long tiles = (max_keys + atc::BKV - 1) / atc::BKV;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= kMaxSplits; ++s) {
+    if (s > 1 && tiles / s < 2) break;
+    const long long work = ctas * s;
+    const long long waves = (work + sms - 1) / sms;
+    const double eff = (double)work / (double)(waves * sms);
+    if (eff > best_eff + 0.04) {
+      best = s;
+      best_eff = eff;
+    }
+  }
+  return best;
+}
+
+// q: map over [rows][H][128]; k, v: maps over the key rows ([rows][H][128]).
+int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const AttnDesc& a, int kv_row0, int n_heads, int n_splits, void* o,
+                        float* o_part, float* lse_part, int* err, cudaStream_t s) {
+  const long long total_rows = (long long)a.n * a.rows_per;
+  if (total_rows == 0) return SFM_OK;
+  atc::Args args{};
+  args.a = a;
+  args.H = n_heads;
+  args.n_splits = n_splits;
+  args.qtiles = (a.rows_per + atc::BQ - 1) / atc::BQ;
+  args.scale_log2 = (float)(1.4426950408889634 / sqrt((double)atc::D));
+  args.total_rows = total_rows;
+  args.kv_row0 = kv_row0;
+  args.o = (__nv_bfloat16*)o;
+  args.o_part = o_part;
+  args.lse_part = lse_part;
+  args.err = err;
+  dim3 grid(a.n * args.qtiles, n_heads, n_splits);
+  cudaFuncSetAttribute(atc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, atc::SMEM);
+  int rc;
+  {
+    ProfScope ps(SFM_PROF_ATTN, s);
+    atc::attn_tc_kernel<<<grid, atc::THREADS, atc::SMEM, s>>>(mq, mk, mv, args);
+    rc = record_cuda(cudaGetLastError());
+  }
+  if (rc || n_splits == 1) return rc;
+  ProfScope ps(SFM_PROF_ATTN_MERGE, s);
+  return launch_attention_merge(o_part, lse_part, o, total_rows, n_heads, n_splits, s);
+}
+
+}  // namespace sfm

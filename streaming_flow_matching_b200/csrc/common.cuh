@@ -74,7 +74,7 @@ int launch_head_euler(const BatchDesc& b, const float* x, const void* g, const v
 int launch_euler(float* z, const float* v, float dtau, long long n, cudaStream_t s);
 
 // GEMM C = A B^T, A [M][K], B [N][K] (both K-contiguous).
-enum Epilogue { EPI_F32 = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_STORE = 3 };
+enum Epilogue { EPI_F32 = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_STORE = 3, EPI_QKV = 4 };
 int launch_gemm(const void* A, const void* B, void* C, int M, int N, int K, int epi, int dtype,
                 cudaStream_t s);
 

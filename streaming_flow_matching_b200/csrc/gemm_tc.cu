@@ -1,0 +1,324 @@
+// Dense projections of f_theta on the 5th-generation tensor cores (tcgen05):
+//   C[M][N] = A[M][K] . B[N][K]^T,  A = activations (bf16), B = weights (bf16,
+//   stored [out][in]), fp32 accumulation in tensor memory.
+//
+// Persistent, warp-specialised CTA (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A tile 128 x 64 and B tile BN x 64 per stage
+//               (128-byte swizzle), STAGES-deep ring of shared-memory stages
+//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=BN, K=16)
+//               into one of two TMEM accumulators and commits to mbarriers
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (thread = row), fused
+//               epilogue, global stores; the other accumulator is being filled
+//               meanwhile
+// Epilogues: EPI_F32 / EPI_STORE / EPI_GELU / EPI_RESID (x += acc, fp32) and
+// EPI_QKV: rotary embedding of q and k in fp32 (rotate-half pairs (i, i+64) of
+// each 128-wide head), q to the Q buffer, k and v to the sessions' cache rows
+// after their valid cache (the current unit's scratch rows).
+#include "gemm_tc.cuh"
+#include "sm100.cuh"
+
+namespace sfm {
+
+using namespace sm100;
+
+namespace gtc {
+
+constexpr int BM = 128, BK = 64;
+constexpr int THREADS = 192;
+
+template <int BN> struct Cfg {
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+};
+
+__device__ __forceinline__ float gelu_tanh(float x) {
+  const float k = 0.7978845608028654f;
+  return 0.5f * x * (1.f + tanhf(k * (x + 0.044715f * x * x * x)));
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = u;
+  }
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a,
+                   const __grid_constant__ CUtensorMap map_b, const __grid_constant__ GemmArgs args) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (args.M + BM - 1) / BM;
+  const int n_tiles = args.N / BN;
+  const int tiles = m_tiles * n_tiles;
+  const int kblocks = args.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&map_a);
+    tma_prefetch(&map_b);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int s = 0;
+      uint32_t ph = 0;
+      int last_parity[8];
+      for (int i = 0; i < C::STAGES; ++i) last_parity[i] = -1;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int m0 = (t % m_tiles) * BM, n0 = (t / m_tiles) * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort, args.err, 0x101)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = base + s * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+          tma_load_2d(sa, &map_a, &full[s], kb * BK, m0);
+          tma_load_2d(sa + C::A_BYTES, &map_b, &full[s], kb * BK, n0);
+          last_parity[s] = (int)ph;
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok)  // unwinding: let the loads already issued land before the CTA exits
+        for (int i = 0; i < C::STAGES; ++i)
+          if (last_parity[i] >= 0) mbar_drain(&full[i], (uint32_t)last_parity[i]);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = idesc_bf16(BM, BN, false, false);
+      int s = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true, issued = false;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[s], ph, abort, args.err, 0x103)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + s * C::STAGE_BYTES;
+          const uint64_t da = sw128_desc(sa, 16, 1024);
+          const uint64_t db = sw128_desc(sa + C::A_BYTES, 16, 1024);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)  // +32 bytes per K=16 step inside the swizzle atom
+            umma_bf16(d, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
+                      (kb | k) != 0 ? 1u : 0u);
+          issued = true;
+          umma_commit(&empty[s]);
+          if (++s == C::STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_ph ^= 1u;
+      }
+      if (!ok && issued) {  // unwinding: wait for the MMAs already issued
+        umma_commit(drain);
+        mbar_drain(drain, 0);
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5, thread = accumulator row) ----------------
+    const int quarter = warp & 3;              // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
+      const int m0 = (t % m_tiles) * BM, n0 = (t / m_tiles) * BN;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_ph, abort, args.err, 0x104))) break;
+      tc_fence_after();
+      const int row = m0 + quarter * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      if (EPI == EPI_QKV) {
+        const int hd = args.hd;
+        const int section = n0 / hd;           // 0 q, 1 k, 2 v (a tile never straddles)
+        for (int hh = 0; hh < BN / 128; ++hh) {
+          const int head = (n0 - section * hd) / 128 + hh;
+          for (int half = 0; half < 2; ++half) {
+            uint32_t ra[32], rb[32];
+            tmem_ld32(tbase + hh * 128 + half * 32, ra);
+            tmem_ld32(tbase + hh * 128 + 64 + half * 32, rb);
+            tmem_ld_wait();
+            if (row >= args.M) continue;
+            float a[32], b[32];
+            if (section < 2) {
+              const float* cs = args.cos_t + (size_t)row * 64 + half * 32;
+              const float* sn = args.sin_t + (size_t)row * 64 + half * 32;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float x = __uint_as_float(ra[i]), y = __uint_as_float(rb[i]);
+                const float c = cs[i], s = sn[i];
+                a[i] = x * c - y * s;
+                b[i] = y * c + x * s;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                a[i] = __uint_as_float(ra[i]);
+                b[i] = __uint_as_float(rb[i]);
+              }
+            }
+            __nv_bfloat16* dst;
+            if (section == 0) {
+              dst = args.q_out + (size_t)row * hd + head * 128;
+            } else {
+              const int sess = row / args.b.n_tok;
+              const int j = row - sess * args.b.n_tok;
+              const long long prow = args.b.base[sess] + args.b.valid[sess] + j;
+              dst = (section == 1 ? args.k_layer : args.v_layer) + prow * hd + head * 128;
+            }
+            store_bf16x32(dst + half * 32, a);
+            store_bf16x32(dst + 64 + half * 32, b);
+          }
+        }
+      } else {
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tbase + c * 32, r);
+          tmem_ld_wait();
+          if (row >= args.M) continue;
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          const int col = n0 + c * 32;
+          if (EPI == EPI_F32) {
+            float4* d = reinterpret_cast<float4*>((float*)args.C + (size_t)row * args.ldc + col);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          } else if (EPI == EPI_RESID) {
+            float4* d = reinterpret_cast<float4*>((float*)args.C + (size_t)row * args.ldc + col);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              float4 x = d[q];
+              x.x += v[4 * q];
+              x.y += v[4 * q + 1];
+              x.z += v[4 * q + 2];
+              x.w += v[4 * q + 3];
+              d[q] = x;
+            }
+          } else {
+            if (EPI == EPI_GELU) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+            }
+            store_bf16x32((__nv_bfloat16*)args.C + (size_t)row * args.ldc + col, v);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_ph ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int BN, int EPI>
+int launch_bn(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,
+              cudaStream_t s) {
+  using C = Cfg<BN>;
+  const int tiles = ((args.M + BM - 1) / BM) * (args.N / BN);
+  const int grid = tiles < sms ? tiles : sms;
+  cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       C::SMEM);
+  gemm_tc_kernel<BN, EPI><<<grid, THREADS, C::SMEM, s>>>(a, b, args);
+  return record_cuda(cudaGetLastError());
+}
+
+}  // namespace gtc
+
+int gemm_tc_block_n(int N, int hd, int epi) {
+  if (epi == EPI_QKV) return (hd % 256 == 0) ? 256 : 128;
+  return (N % 256 == 0) ? 256 : 128;
+}
+
+int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,
+                   cudaStream_t s) {
+  if (args.M <= 0) return SFM_OK;
+  const int bn = gemm_tc_block_n(args.N, args.hd, args.epi);
+  if (args.N % bn || args.K % gtc::BK || args.K <= 0) return SFM_EUNSUPPORTED;
+  if (args.epi == EPI_QKV && (args.hd % bn || args.N != 3 * args.hd)) return SFM_EUNSUPPORTED;
+#define SFM_GTC(BN_, E)                                          \
+  if (bn == BN_ && args.epi == E) return gtc::launch_bn<BN_, E>(a, b, args, sms, s);
+  SFM_GTC(256, EPI_F32)
+  SFM_GTC(256, EPI_GELU)
+  SFM_GTC(256, EPI_RESID)
+  SFM_GTC(256, EPI_STORE)
+  SFM_GTC(256, EPI_QKV)
+  SFM_GTC(128, EPI_F32)
+  SFM_GTC(128, EPI_GELU)
+  SFM_GTC(128, EPI_RESID)
+  SFM_GTC(128, EPI_STORE)
+  SFM_GTC(128, EPI_QKV)
+#undef SFM_GTC
+  return SFM_EINVAL;
+}
+
+}  // namespace sfm

@@ -1,0 +1,31 @@
+// tcgen05 GEMM launch interface.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace sfm {
+
+struct GemmArgs {
+  int M, N, K;
+  int epi;               // Epilogue
+  void* C;               // output (EPI_F32 / EPI_STORE / EPI_GELU) or fp32 residual (EPI_RESID)
+  int ldc;
+  int* err;              // device error word (bounded-wait timeouts)
+  // EPI_QKV
+  const float* cos_t;    // [M][64]
+  const float* sin_t;
+  __nv_bfloat16* q_out;  // [M][hd]
+  __nv_bfloat16* k_layer;  // cache pool rows of this layer, [rows][hd]
+  __nv_bfloat16* v_layer;
+  int hd;
+  BatchDesc b;
+};
+
+// Block N the kernel uses for a problem (128 or 256).
+int gemm_tc_block_n(int N, int hd, int epi);
+// A: tensor map over [M_alloc][K] bf16, box {64, 128}; B: over [N][K], box {64, block_n}.
+int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,
+                   cudaStream_t s);
+
+}  // namespace sfm

@@ -136,6 +136,12 @@ class Performer:
         L.check(L.lib.sfm_fm_solve_batched(self._h, n, s, zp, t, len(taus), _stream()),
                 "sfm_fm_solve_batched")
 
+    def check_device_error(self):
+        """Synchronises and returns the handle's device error word (0 = no kernel problem)."""
+        code = C.c_int()
+        L.check(L.lib.sfm_check_device_error(self._h, C.byref(code)), "sfm_check_device_error")
+        return code.value
+
     def close(self):
         if self._h:
             L.lib.sfm_destroy(self._h)
@@ -169,6 +175,26 @@ def attention(q, k, v, out=None, workspace=None):
 
 def attention_workspace_bytes(n_q, n_kv, n_heads, head_dim, dtype=torch.bfloat16):
     return L.lib.sfm_attention_workspace_bytes(n_q, n_kv, n_heads, head_dim, _DT[dtype])
+
+
+_LINEAR = {"f32": L.SFM_LINEAR_F32, "out": L.SFM_LINEAR_OUT, "gelu": L.SFM_LINEAR_GELU,
+           "resid": L.SFM_LINEAR_RESID}
+
+
+def linear(x, w, y=None, epilogue="f32"):
+    """y = x W^T (w stored [out][in]); epilogue f32 | out | gelu | resid (y += x W^T, fp32 y)."""
+    dt = _DT[x.dtype]
+    _need(x, x.dtype, "x")
+    _need(w, x.dtype, "w")
+    M, K = x.shape
+    N = w.shape[0]
+    if y is None:
+        odt = x.dtype if epilogue in ("out", "gelu") else torch.float32
+        y = torch.zeros(M, N, dtype=odt, device=x.device)
+    _need(y, y.dtype, "y", (M, N))
+    L.check(L.lib.sfm_linear(_ptr(x), _ptr(w), _ptr(y), M, N, K, _LINEAR[epilogue], dt, _stream()),
+            "sfm_linear")
+    return y
 
 
 def euler_update(z, v, dtau):

@@ -156,6 +156,27 @@ def test_attention_sweep_sampled_rows(cuda_device, n_kv):
     assert e <= BF16_TOL, e
 
 
+@pytest.mark.parametrize("n_kv", [512, 20000])
+def test_attention_max_jump_in_some_rows_only(cuda_device, n_kv):
+    # A few rows (one lane in each of several warps) meet a key aligned with their
+    # query in a later key tile: their running max jumps by far more than 2^8 while
+    # the rest of the warp's rows do not, so the online-softmax rescale of O is
+    # needed by only some rows of a warp.
+    from streaming_flow_matching_b200 import attention
+    g = torch.Generator().manual_seed(21)
+    n_q, H = 128, 2
+    q = torch.randn(n_q, H, 128, generator=g)
+    k = 0.1 * torch.randn(n_kv, H, 128, generator=g)
+    v = torch.randn(n_kv, H, 128, generator=g)
+    for i, r in enumerate([3, 40, 77, 101]):
+        k[300 + i] = 2.0 * q[r]
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    o = attention(q.cuda(), k.cuda(), v.cuda())
+    torch.cuda.synchronize()
+    e = rel_l2(o.float().cpu().numpy(), O.attention(q, k, v))
+    assert e <= BF16_TOL, e
+
+
 def test_attention_fp32_matches_oracle(cuda_device):
     from streaming_flow_matching_b200 import attention
     q, k, v = S.make_qkv(68, 452, 4, 64, dtype="fp32")

@@ -345,7 +345,7 @@ def run_ours(args, w):
         contraction_flop = args.steps * w.n_steps * fl["per_euler_step"]
         ap_ms, ap_n = prof["append"]
         append_gbs = append_bytes(w) / (ap_ms / max(ap_n, 1) / 1e3) / 1e9 if ap_n else None
-        attn_src = os.path.join(ROOT, "streaming_flow_matching_b200", "csrc", "attn_simt.cu")
+        attn_src = os.path.join(ROOT, "streaming_flow_matching_b200", "csrc", "attn_tc.cu")
         traffic = traffic_for(attn_src)
         unit_ms = ms_max / args.steps
         line = {
@@ -358,7 +358,7 @@ def run_ours(args, w):
             "unit_latency_ms": unit_ms,
             "e2e": e2e,
             "gpu_launches": launches,
-            "roofline": {"kernel": "attention (flash, split-KV)", "bound": "tensor",
+            "roofline": {"kernel": "attn_tc_kernel (tcgen05 flash attention, split-KV)", "bound": "tensor",
                          "achieved": attn_tflops, "peak": pk["bf16_sustained"],
                          "unit": "TFLOP/s", "frac": attn_tflops / pk["bf16_sustained"],
                          "traffic": traffic,

@@ -17,7 +17,6 @@ struct AttnDesc {
   int nkeys[kMaxBatch];
 };
 
-int attention_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads);
 size_t attention_workspace_bytes(long long rows, int n_heads, int n_splits);
 int launch_attention(const AttnDesc& a, const void* q, const void* k, const void* v, void* o,
                      int n_heads, int head_dim, int dtype, int n_splits, float* o_part,

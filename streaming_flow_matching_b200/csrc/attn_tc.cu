@@ -241,26 +241,29 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       tc_fence_after();
-      float s[128];
-      {
-        uint32_t u[32];
+      // S row: 4 x 32 columns, one wait for all four loads
+      uint32_t u[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tmem + lane_base + (uint32_t)((j & 1) * 128 + c * 32), u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(u[i]);
-        }
-      }
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tmem + lane_base + (uint32_t)((j & 1) * 128 + c * 32), u[c]);
+      tmem_ld_wait();
+      float* sv = reinterpret_cast<float*>(&u[0][0]);
       const int kvalid = nkeys - (t0 + j) * BKV;         // > 0
-      float mx = -INFINITY;
+      if (kvalid < BKV) {                                // partial tile only (CTA-uniform)
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        float x = s[i] * args.scale_log2;
-        if (i >= kvalid) x = -INFINITY;
-        s[i] = x;
-        mx = fmaxf(mx, x);
+        for (int i = 0; i < 128; ++i)
+          if (i >= kvalid) sv[i] = -INFINITY;
       }
+      // row max of the raw logits (the scale is positive), four independent chains
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int i = 0; i < 128; i += 4) {
+        m4[0] = fmaxf(m4[0], sv[i]);
+        m4[1] = fmaxf(m4[1], sv[i + 1]);
+        m4[2] = fmaxf(m4[2], sv[i + 2]);
+        m4[3] = fmaxf(m4[3], sv[i + 3]);
+      }
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * args.scale_log2;
       if (j > 0) {
         // PV_{j-1} must be complete before O is rescaled or P is overwritten
         if (!__all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((j - 1) & 1), abort, args.err, 0x208))) {
@@ -276,28 +279,30 @@ __global__ void __launch_bounds__(THREADS, 1)
         m = mx;
       } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
         const float m_new = fmaxf(m, mx);
-        const float alpha = exp2f(m - m_new);
+        const float alpha = ex2_approx(m - m_new);
         l *= alpha;
         m = m_new;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t u[32];
-          tmem_ld32(tmem + lane_base + COL_O + c * 32, u);
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + COL_O + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st32(tmem + lane_base + COL_O + c * 32, u);
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem + lane_base + COL_O + c * 32, o);
         }
         tmem_st_wait();
       }
-      // P = exp2(x - m) as bf16 into the swizzled K-major P tile (two 64-key halves)
+      // P = 2^(s * scale - m) as bf16 into the swizzled K-major P tile (two 64-key halves)
+      const float neg_m = -m, sc = args.scale_log2;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         float p[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          p[e] = exp2f(s[c * 8 + e] - m);
-          l += p[e];
+          p[e] = ex2_approx(fmaf(sv[c * 8 + e], sc, neg_m));
+          l4[e & 3] += p[e];
         }
         uint4 w;
         w.x = pack_bf16x2(p[0], p[1]);
@@ -307,6 +312,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int half = c >> 3, chunk = c & 7;
         *reinterpret_cast<uint4*>(prow + half * HALF + ((chunk ^ (r & 7)) << 4)) = w;
       }
+      l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       if (kvalid < BKV) {
         // zero the V rows of the partial tile past the key range once the tile has landed
         const int vs = j % VST;

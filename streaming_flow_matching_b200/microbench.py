@@ -3,6 +3,7 @@
   python -m streaming_flow_matching_b200.microbench attention --n-kv 16800 [--n-q 924 --heads 24]
   python -m streaming_flow_matching_b200.microbench append [--layers 28 --units 1]
   python -m streaming_flow_matching_b200.microbench euler [--n 268435456]
+  python -m streaming_flow_matching_b200.microbench linear --m 924 --n 12288 --k 3072 [--epilogue gelu]
   python -m streaming_flow_matching_b200.microbench sweep      # attention + append sweep
 
 Inputs are seeded and larger than L2 where the case allows; each timing is
@@ -24,7 +25,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 import sfm_synth as S  # noqa: E402
-from streaming_flow_matching_b200 import Performer, attention, attention_workspace_bytes, euler_update  # noqa: E402
+from streaming_flow_matching_b200 import (Performer, attention, attention_workspace_bytes,  # noqa: E402
+                                          euler_update, linear)
 
 
 def _peaks():
@@ -82,6 +84,20 @@ def bench_append(layers, units, warmup, reps):
             "gb_s": gbs, "frac_of_hbm": gbs / hbm, "peak_source": src}
 
 
+def bench_linear(m, n, k, epilogue, warmup, reps):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(6)
+    x = torch.randn(m, k, generator=g, device="cuda").to(torch.bfloat16)
+    w = (0.02 * torch.randn(n, k, generator=g, device="cuda")).to(torch.bfloat16)
+    y = torch.zeros(m, n, device="cuda",
+                    dtype=torch.bfloat16 if epilogue in ("out", "gelu") else torch.float32)
+    ms = _time(lambda: linear(x, w, y, epilogue), warmup, reps)
+    _, bf16, src = _peaks()
+    tf = 2.0 * m * n * k / (ms / 1e3) / 1e12
+    return {"case": "linear", "m": m, "n": n, "k": k, "epilogue": epilogue, "ms": ms,
+            "tflops": tf, "frac_of_bf16_burst": tf / bf16, "peak_source": src}
+
+
 def bench_euler(n, warmup, reps):
     g = torch.Generator(device="cuda")
     g.manual_seed(4)
@@ -96,7 +112,10 @@ def bench_euler(n, warmup, reps):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attention", "append", "euler", "sweep"])
+    ap.add_argument("case", choices=["attention", "append", "euler", "linear", "sweep"])
+    ap.add_argument("--m", type=int, default=924)
+    ap.add_argument("--k", type=int, default=3072)
+    ap.add_argument("--epilogue", default="gelu")
     ap.add_argument("--n-q", type=int, default=924)
     ap.add_argument("--n-kv", type=int, default=57600 + 924)
     ap.add_argument("--heads", type=int, default=24)
@@ -114,7 +133,12 @@ def main():
         out.append(bench_append(a.layers, a.units, a.warmup, a.reps))
     elif a.case == "euler":
         out.append(bench_euler(a.n, a.warmup, a.reps))
+    elif a.case == "linear":
+        out.append(bench_linear(a.m, a.n, a.k, a.epilogue, a.warmup, a.reps))
     else:
+        for m, n, k, e in [(924, 9216, 3072, "f32"), (924, 3072, 3072, "resid"),
+                           (924, 12288, 3072, "gelu"), (924, 3072, 12288, "resid")]:
+            out.append(bench_linear(m, n, k, e, a.warmup, a.reps))
         for n_kv in S.ATTN_SWEEP_TOKENS:
             out.append(bench_attention(a.n_q, n_kv + a.n_q, a.heads, a.warmup, a.reps))
         out.append(bench_append(1, 1, a.warmup, a.reps))

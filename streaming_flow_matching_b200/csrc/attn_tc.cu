@@ -5,20 +5,24 @@
 // key of the current unit, so O = softmax(Q K^T / sqrt(D)) V over one key
 // range per session, D = 128.
 //
-// One CTA = one (session, head, 128-query tile, key split); 192 threads:
-//   warp 0      TMA producer: Q tile once; K tiles (128 keys x 128 dims) in a
-//               3-stage ring, V tiles in a 2-stage ring (128-byte swizzle)
-//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma:
-//                 S_j = Q K_j^T      (M=128, N=128 keys, K=128 dims) into one of
-//                                    two TMEM S buffers, issued two tiles ahead
-//                 O  += P_j V_j      (M=128, N=128 dims, K=128 keys; V as an
-//                                    MN-major operand) into the TMEM O buffer
-//   warps 2-5   softmax, thread = query row: tcgen05.ld of its S row, online
-//               softmax in the exp2 domain, P (bf16) written to shared memory in
-//               the swizzled K-major layout, O rescaled in TMEM only when the
-//               running max grows by more than 2^8 (otherwise the stale max is
-//               kept; P <= 2^8 stays exact in fp32 sums), final O / l written
-//               as bf16 (one split) or as fp32 partials + log2-sum-exp (several).
+// One CTA = one (session, head, 256-query block, key split): two 128-row
+// query tiles A and B share every K/V tile.  320 threads:
+//   warp 0      TMA producer: both Q tiles once; K tiles (128 keys x 128 dims)
+//               in a 3-stage ring, V tiles in a 2-stage ring (128-byte swizzle)
+//   warp 1      TMEM allocator; lane 0 issues tcgen05.mma, alternating tiles:
+//                 S_t = Q_t K_j^T   (M=128, N=128 keys, K=128 dims), smem x smem
+//                 O_t += P_t V_j    (M=128, N=128 dims, K=128 keys), P from TMEM,
+//                                   V from smem as an MN-major operand
+//               S_t of the next key tile is issued once O_t's P V has completed
+//               (P_t aliases S_t in TMEM).
+//   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B (thread = query
+//               row): two passes over the S row in TMEM (row max, then
+//               p = 2^(s scale - m)), P written back to TMEM as packed bf16;
+//               O rescaled in TMEM only when a row's running max grows by more
+//               than 2^8 (decided per warp: the TMEM accesses are collective);
+//               final O / l written as bf16 (one split) or as fp32 partials +
+//               log2-sum-exp (several splits).
+// TMEM columns: tile A S/P [0,128) O [128,256); tile B S/P [256,384) O [384,512).
 // The last, partial key tile is masked in S, and its V rows past the key range
 // are zeroed in shared memory before P V, so rows outside the range never
 // contribute (whatever they hold).
@@ -33,26 +37,25 @@ using namespace sm100;
 
 namespace atc {
 
-constexpr int BQ = 128, BKV = 128, D = 128;
-constexpr int THREADS = 192;
+constexpr int BQ = 128, QT = 2, BKV = 128, D = 128;
+constexpr int ROWS = BQ * QT;               // query rows per CTA
+constexpr int THREADS = 320;
 constexpr int KST = 3, VST = 2;
-constexpr int HALF = 128 * 64 * 2;        // one [128 rows][64 cols] bf16 swizzle tile: 16 KB
-constexpr int TILE = 2 * HALF;            // [128][128] bf16: 32 KB
-constexpr int OFF_Q = 0;
-constexpr int OFF_P = OFF_Q + TILE;
-constexpr int OFF_K = OFF_P + TILE;
+constexpr int HALF = 128 * 64 * 2;          // one [128 rows][64 cols] bf16 swizzle tile: 16 KB
+constexpr int TILE = 2 * HALF;              // [128][128] bf16: 32 KB
+constexpr int OFF_Q = 0;                    // Q_A, Q_B
+constexpr int OFF_K = OFF_Q + QT * TILE;
 constexpr int OFF_V = OFF_K + KST * TILE;
 constexpr int OFF_BAR = OFF_V + VST * TILE;      // 229376
 constexpr int SMEM = OFF_BAR + 256 + 1024;
-constexpr uint32_t TMEM_COLS = 512;               // S0 | S1 | O
-constexpr uint32_t COL_O = 256;
+constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
 struct Args {
   AttnDesc a;
   int H;
   int n_splits;
-  int qtiles;
+  int qtiles;                  // 256-row query blocks per session
   float scale_log2;
   long long total_rows;
   int kv_row0;                 // row offset of this layer inside the K/V tensor maps
@@ -62,6 +65,8 @@ struct Args {
   int* err;
 };
 
+// 10 warps: two of the four SM sub-partitions hold three warps, which caps a
+// thread at 16384 / (3 * 32) registers -- the launch bound makes ptxas respect it.
 __global__ void __launch_bounds__(THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ Args args) {
@@ -75,19 +80,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* k_empty = k_full + KST;
   uint64_t* v_full = k_empty + KST;
   uint64_t* v_empty = v_full + VST;
-  uint64_t* s_full = v_empty + VST;   // [2]
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 1;
-  uint64_t* drain = o_done + 1;
+  uint64_t* s_full = v_empty + VST;   // [QT]
+  uint64_t* p_full = s_full + QT;     // [QT]
+  uint64_t* o_done = p_full + QT;     // [QT]
+  uint64_t* drain = o_done + QT;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sess = blockIdx.x / args.qtiles;
-  const int qt = blockIdx.x - sess * args.qtiles;
+  const int qb = blockIdx.x - sess * args.qtiles;
   const int h = blockIdx.y, split = blockIdx.z;
-  const long long row0 = (long long)sess * args.a.rows_per + qt * BQ;
-  const int q_rows = min(BQ, args.a.rows_per - qt * BQ);
+  const long long row0 = (long long)sess * args.a.rows_per + (long long)qb * ROWS;
   const int nkeys = args.a.nkeys[sess];
   const long long kbase = args.a.kbase[sess];
   const int ntiles = (nkeys + BKV - 1) / BKV;
@@ -106,10 +110,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    for (int t = 0; t < QT; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_done[t], 1);
+    }
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
@@ -135,9 +140,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int i = 0; i < KST; ++i) kp[i] = -1;
       for (int i = 0; i < VST; ++i) vp[i] = -1;
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, TILE);
-      tma_load_3d(base + OFF_Q, &map_q, q_full, 0, h, (int)row0);
-      tma_load_3d(base + OFF_Q + HALF, &map_q, q_full, 64, h, (int)row0);
+      mbar_arrive_expect_tx(q_full, QT * TILE);
+      for (int t = 0; t < QT; ++t) {
+        tma_load_3d(base + OFF_Q + t * TILE, &map_q, q_full, 0, h, (int)(row0 + t * BQ));
+        tma_load_3d(base + OFF_Q + t * TILE + HALF, &map_q, q_full, 64, h, (int)(row0 + t * BQ));
+      }
       auto load_k = [&](int i) -> bool {   // i: tile index relative to t0
         const int s = i % KST;
         const uint32_t par = (uint32_t)((i / KST) & 1);
@@ -160,8 +167,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         vp[s] = (int)par;
         return true;
       };
-      // order of need by the MMA issuer: S_0, S_1, then per j: PV_j, S_{j+2}
-      if (ok && T > 0) ok = load_k(0);
+      // order of need by the MMA issuer: S(0); then per j: P V (V_j), S(j+1) (K_{j+1})
+      if (ok) ok = load_k(0);
       if (ok && T > 1) ok = load_k(1);
       for (int j = 0; j < T && ok; ++j) {
         ok = load_v(j);
@@ -181,12 +188,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr uint32_t idesc_s = idesc_bf16(BQ, BKV, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(BQ, D, false, true);
       bool ok = mbar_wait(q_full, 0, abort, args.err, 0x203), issued = false;
-      auto issue_s = [&](int i) -> bool {
-        const int s = i % KST;
-        if (!mbar_wait(&k_full[s], (uint32_t)((i / KST) & 1), abort, args.err, 0x204)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)((i & 1) * 128);
-        const uint32_t qa = base + OFF_Q, ka = base + OFF_K + s * TILE;
+      auto issue_s = [&](int t, int ks) {   // S_t = Q_t K^T from K stage ks
+        const uint32_t qa = base + OFF_Q + t * TILE, ka = base + OFF_K + ks * TILE;
+        const uint32_t d = tmem + (uint32_t)(t * 256);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t sub = (uint32_t)(kk >> 2) * HALF;
@@ -194,33 +198,58 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint64_t db = sw128_desc(ka + sub, 16, 1024) + (uint64_t)(2 * (kk & 3));
           umma_bf16(d, da, db, idesc_s, kk > 0 ? 1u : 0u);
         }
+        umma_commit(&s_full[t]);
         issued = true;
-        umma_commit(&k_empty[s]);
-        umma_commit(&s_full[i & 1]);
-        return true;
       };
-      if (ok && T > 0) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
+      if (ok && (ok = mbar_wait(&k_full[0], 0, abort, args.err, 0x204))) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(&k_empty[0]);
+      }
+      // per key tile j: P_A V, S_A(j+1), P_B V, S_B(j+1) -- tile A never waits on tile B,
+      // so the two softmax warpgroups run half a period apart
       for (int j = 0; j < T && ok; ++j) {
         const int vs = j % VST;
-        if (!mbar_wait(p_full, (uint32_t)(j & 1), abort, args.err, 0x205) ||
-            !mbar_wait(&v_full[vs], (uint32_t)((j / VST) & 1), abort, args.err, 0x206)) {
+        const bool more = j + 1 < T;
+        const int ks = (j + 1) % KST;
+        if (!mbar_wait(&v_full[vs], (uint32_t)((j / VST) & 1), abort, args.err, 0x206)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        const uint32_t pa = base + OFF_P, va = base + OFF_V + vs * TILE;
+        const uint32_t va = base + OFF_V + vs * TILE;
+        for (int t = 0; t < QT && ok; ++t) {
+          if (!mbar_wait(&p_full[t], (uint32_t)(j & 1), abort, args.err, 0x205)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t pa = tmem + (uint32_t)(t * 256);          // P_t: packed bf16, 64 columns
+          const uint32_t d = tmem + (uint32_t)(t * 256 + 128);     // O_t
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t da = sw128_desc(pa + (uint32_t)(kk >> 2) * HALF, 16, 1024) +
-                              (uint64_t)(2 * (kk & 3));
-          // V as MN-major B: 64-dim halves HALF bytes apart, 16 keys = 2048 B per K step
-          const uint64_t db = sw128_desc(va + (uint32_t)kk * 2048u, HALF, 1024);
-          umma_bf16(tmem + COL_O, da, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            // V as MN-major B: 64-dim halves HALF bytes apart, 16 keys = 2048 B per K step
+            const uint64_t db = sw128_desc(va + (uint32_t)kk * 2048u, HALF, 1024);
+            umma_bf16_tmem_a(d, pa + (uint32_t)(kk * 8), db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&o_done[t]);
+          if (t == QT - 1) umma_commit(&v_empty[vs]);
+          if (more) {
+            if (t == 0 &&
+                !mbar_wait(&k_full[ks], (uint32_t)(((j + 1) / KST) & 1), abort, args.err, 0x204)) {
+              ok = false;
+              break;
+            }
+            // S_t(j+1) overwrites P_t(j): wait until O_t's P V of this tile has completed
+            if (!mbar_wait(&o_done[t], (uint32_t)(j & 1), abort, args.err, 0x20B)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(t, ks);
+            if (t == QT - 1) umma_commit(&k_empty[ks]);
+          }
         }
-        umma_commit(&v_empty[vs]);
-        umma_commit(o_done);
-        if (j + 2 < T) ok = issue_s(j + 2);
       }
       if (!ok && issued) {
         umma_commit(drain);
@@ -228,53 +257,61 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else {
-    // ---------------- softmax + output (warps 2..5, thread = query row) ----------------
+    // ---------------- softmax + output (thread = query row of tile t) ----------------
+    const int t = (warp - 2) >> 2;                        // 0: tile A, 1: tile B
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;                    // row inside the tile
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t col_s = (uint32_t)(t * 256), col_o = col_s + 128;
+    const int q_rows = min(BQ, args.a.rows_per - qb * ROWS - t * BQ);   // may be <= 0
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* prow = smem + OFF_P + r * 128;
+    const float sc = args.scale_log2;
     for (int j = 0; j < T && ok; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (uint32_t)((j >> 1) & 1), abort, args.err, 0x207))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], (uint32_t)(j & 1), abort, args.err, 0x207))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // S row: 4 x 32 columns, one wait for all four loads
-      uint32_t u[4][32];
+      const int kvalid = nkeys - (t0 + j) * BKV;         // > 0; < BKV only on the last tile
+      if (kvalid < BKV) {
+        // partial tile (CTA-uniform): overwrite the logits past the key range with -inf
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(tmem + lane_base + (uint32_t)((j & 1) * 128 + c * 32), u[c]);
-      tmem_ld_wait();
-      float* sv = reinterpret_cast<float*>(&u[0][0]);
-      const int kvalid = nkeys - (t0 + j) * BKV;         // > 0
-      if (kvalid < BKV) {                                // partial tile only (CTA-uniform)
+        for (int c = 0; c < 4; ++c) {
+          if (c * 32 + 32 <= kvalid) continue;
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_base + col_s + c * 32, u);
+          tmem_wait_ld(u);
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i >= kvalid) sv[i] = -INFINITY;
-      }
-      // row max of the raw logits (the scale is positive), four independent chains
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int i = 0; i < 128; i += 4) {
-        m4[0] = fmaxf(m4[0], sv[i]);
-        m4[1] = fmaxf(m4[1], sv[i + 1]);
-        m4[2] = fmaxf(m4[2], sv[i + 2]);
-        m4[3] = fmaxf(m4[3], sv[i + 3]);
-      }
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * args.scale_log2;
-      if (j > 0) {
-        // PV_{j-1} must be complete before O is rescaled or P is overwritten
-        if (!__all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((j - 1) & 1), abort, args.err, 0x208))) {
-          ok = false;
-          break;
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i >= kvalid) u[i] = __float_as_uint(-INFINITY);
+          tmem_st32(tmem + lane_base + col_s + c * 32, u);
         }
-        tc_fence_after();
+        tmem_st_wait();
       }
-      // tcgen05.ld/st are warp-collective: the rescale decision is taken per warp
-      // (any row needing it rescales the whole warp; a row whose max did not grow
-      // gets alpha = 1).
+      // pass 1: row max of the raw logits (the scale is positive); the load of the
+      // next 32-column chunk overlaps the max over the current one
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      {
+        uint32_t u[2][32];
+        tmem_ld32(tmem + lane_base + col_s, u[0]);
+        tmem_wait_ld(u[0]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c + 1 < 4) tmem_ld32(tmem + lane_base + col_s + (c + 1) * 32, u[(c + 1) & 1]);
+          const float* sv = reinterpret_cast<const float*>(u[c & 1]);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            m4[0] = fmaxf(m4[0], sv[i]);
+            m4[1] = fmaxf(m4[1], sv[i + 1]);
+            m4[2] = fmaxf(m4[2], sv[i + 2]);
+            m4[3] = fmaxf(m4[3], sv[i + 3]);
+          }
+          if (c + 1 < 4) tmem_wait_ld(u[(c + 1) & 1]);
+        }
+      }
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
+      // O_t's previous P V has completed (S_t(j) was issued after it), so O_t may be rescaled
       if (j == 0) {
         m = mx;
       } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
@@ -285,71 +322,78 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_base + COL_O + c * 32, o);
-          tmem_ld_wait();
+          tmem_ld32(tmem + lane_base + col_o + c * 32, o);
+          tmem_wait_ld(o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + lane_base + COL_O + c * 32, o);
+          tmem_st32(tmem + lane_base + col_o + c * 32, o);
         }
-        tmem_st_wait();
       }
-      // P = 2^(s * scale - m) as bf16 into the swizzled K-major P tile (two 64-key halves)
-      const float neg_m = -m, sc = args.scale_log2;
+      // pass 2: p = 2^(s scale - m) as packed bf16 pairs written over the S row:
+      // keys [32 c, 32 c + 32) -> P columns [16 c, 16 c + 16), which hold S columns
+      // already read (chunk c itself or chunk c - 1); the next chunk's load overlaps
+      const float neg_m = -m;
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        uint32_t u[2][32];
+        tmem_ld32(tmem + lane_base + col_s, u[0]);
+        tmem_wait_ld(u[0]);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float p[8];
+        for (int c = 0; c < 4; ++c) {
+          if (c + 1 < 4) tmem_ld32(tmem + lane_base + col_s + (c + 1) * 32, u[(c + 1) & 1]);
+          const float* sv = reinterpret_cast<const float*>(u[c & 1]);
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = ex2_approx(fmaf(sv[c * 8 + e], sc, neg_m));
-          l4[e & 3] += p[e];
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2_approx(fmaf(sv[2 * i], sc, neg_m));
+            const float p1 = ex2_approx(fmaf(sv[2 * i + 1], sc, neg_m));
+            l4[(2 * i) & 3] += p0;
+            l4[(2 * i + 1) & 3] += p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tmem + lane_base + col_s + c * 16, pk);
+          if (c + 1 < 4) tmem_wait_ld(u[(c + 1) & 1]);
         }
-        uint4 w;
-        w.x = pack_bf16x2(p[0], p[1]);
-        w.y = pack_bf16x2(p[2], p[3]);
-        w.z = pack_bf16x2(p[4], p[5]);
-        w.w = pack_bf16x2(p[6], p[7]);
-        const int half = c >> 3, chunk = c & 7;
-        *reinterpret_cast<uint4*>(prow + half * HALF + ((chunk ^ (r & 7)) << 4)) = w;
       }
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-      if (kvalid < BKV) {
-        // zero the V rows of the partial tile past the key range once the tile has landed
+      tmem_st_wait();
+      if (t == 0 && kvalid < BKV) {
+        // zero the V rows of the partial tile past the key range once the tile has
+        // landed (tile A's warps; both P V products are issued after tile A's P is ready)
         const int vs = j % VST;
         if (!__all_sync(0xffffffffu, mbar_wait(&v_full[vs], (uint32_t)((j / VST) & 1), abort, args.err, 0x209))) {
           ok = false;
           break;
         }
-      }
-      if (kvalid < BKV && r >= kvalid) {
-        const int vs = j % VST;
-        uint4* v0 = reinterpret_cast<uint4*>(smem + OFF_V + vs * TILE + r * 128);
-        uint4* v1 = reinterpret_cast<uint4*>(smem + OFF_V + vs * TILE + HALF + r * 128);
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        if (r >= kvalid) {
+          uint4* v0 = reinterpret_cast<uint4*>(smem + OFF_V + vs * TILE + r * 128);
+          uint4* v1 = reinterpret_cast<uint4*>(smem + OFF_V + vs * TILE + HALF + r * 128);
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          v0[q] = z;
-          v1[q] = z;
+          for (int q = 0; q < 8; ++q) {
+            v0[q] = z;
+            v1[q] = z;
+          }
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[t]);
     }
     // ---- output ----
     if (ok && T > 0) {
-      if (!__all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)((T - 1) & 1), abort, args.err, 0x20A))) ok = false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], (uint32_t)((T - 1) & 1), abort, args.err, 0x20A))) ok = false;
       tc_fence_after();
     }
-    const long long grow = row0 + r;
+    const long long grow = row0 + t * BQ + r;
     const long long ld = (long long)args.H * D;
     const bool have = ok && T > 0 && l > 0.f;
     const float inv = have ? 1.f / l : 0.f;
     for (int c = 0; c < 4; ++c) {
       uint32_t u[32];
       if (T > 0) {
-        tmem_ld32(tmem + lane_base + COL_O + c * 32, u);
-        tmem_ld_wait();
+        tmem_ld32(tmem + lane_base + col_o + c * 32, u);
+        tmem_wait_ld(u);
       }
       if (r >= q_rows) continue;
       float o[32];
@@ -385,7 +429,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads,
                         int sms) {
-  const long long ctas = (long long)n_sessions * ((rows_per_session + atc::BQ - 1) / atc::BQ) * n_heads;
+  const long long ctas = (long long)n_sessions * ((rows_per_session + atc::ROWS - 1) / atc::ROWS) * n_heads;
   const long long tiles = (max_keys + atc::BKV - 1) / atc::BKV;
   int best = 1;
   double best_eff = 0.0;
@@ -412,7 +456,7 @@ int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   args.a = a;
   args.H = n_heads;
   args.n_splits = n_splits;
-  args.qtiles = (a.rows_per + atc::BQ - 1) / atc::BQ;
+  args.qtiles = (a.rows_per + atc::ROWS - 1) / atc::ROWS;
   args.scale_log2 = (float)(1.4426950408889634 / sqrt((double)atc::D));
   args.total_rows = total_rows;
   args.kv_row0 = kv_row0;

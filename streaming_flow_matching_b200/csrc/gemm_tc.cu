@@ -198,7 +198,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t ra[32], rb[32];
             tmem_ld32(tbase + hh * 128 + half * 32, ra);
             tmem_ld32(tbase + hh * 128 + 64 + half * 32, rb);
-            tmem_ld_wait();
+            tmem_wait_ld(ra);
+            reg_fence(rb);
             if (row >= args.M) continue;
             float a[32], b[32];
             if (section < 2) {
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
           tmem_ld32(tbase + c * 32, r);
-          tmem_ld_wait();
+          tmem_wait_ld(r);
           if (row >= args.M) continue;
           float v[32];
 #pragma unroll

@@ -150,11 +150,11 @@ int make_b_map(CUtensorMap* m, const void* p, int n, int k, int block_n) {
   return make_tmap_bf16(m, p, 2, dims, strides, box);
 }
 
-// rows of [rows][H][128] bf16 (queries, or keys / values), box 128 rows x 64 dims of one head
-int make_rows_map(CUtensorMap* m, const void* p, long long rows, int heads) {
+// rows of [rows][H][128] bf16 (queries, or keys / values), box box_rows x 64 dims of one head
+int make_rows_map(CUtensorMap* m, const void* p, long long rows, int heads, int box_rows) {
   const uint64_t dims[3] = {128, (uint64_t)heads, (uint64_t)rows};
   const uint64_t strides[2] = {256, (uint64_t)heads * 256};
-  const uint32_t box[3] = {64, 1, 128};
+  const uint32_t box[3] = {64, 1, (uint32_t)box_rows};
   return make_tmap_bf16(m, p, 3, dims, strides, box);
 }
 
@@ -378,11 +378,13 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
   if (!rc && h->has_weights && cfg->dtype == SFM_DTYPE_BF16) {
     const int L_ = cfg->n_layers, d_ = cfg->d_model, hd_ = h->hd, F_ = cfg->d_mlp;
     rc = make_a_map(&h->map_xn, h->xn, (long long)M, d_);
-    if (!rc) rc = make_rows_map(&h->map_q, h->q, (long long)M, cfg->n_heads);
+    if (!rc) rc = make_rows_map(&h->map_q, h->q, (long long)M, cfg->n_heads, kAttnQBoxRows);
     if (!rc && cfg->pool_tokens > 0)
-      rc = make_rows_map(&h->map_kpool, h->k_pool, (long long)L_ * cfg->pool_tokens, cfg->n_heads);
+      rc = make_rows_map(&h->map_kpool, h->k_pool, (long long)L_ * cfg->pool_tokens, cfg->n_heads,
+                         kAttnKVBoxRows);
     if (!rc && cfg->pool_tokens > 0)
-      rc = make_rows_map(&h->map_vpool, h->v_pool, (long long)L_ * cfg->pool_tokens, cfg->n_heads);
+      rc = make_rows_map(&h->map_vpool, h->v_pool, (long long)L_ * cfg->pool_tokens, cfg->n_heads,
+                         kAttnKVBoxRows);
     if (!rc) rc = make_a_map(&h->map_ao, h->ao, (long long)M, hd_);
     if (!rc) rc = make_a_map(&h->map_hmlp, h->hmlp, (long long)M, F_);
     h->map_wqkv.resize(L_);
@@ -577,9 +579,9 @@ int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q,
     lse_part = o_part + (size_t)splits * n_q * n_heads * 128;
   }
   CUtensorMap mq, mk, mv;
-  int rc = make_rows_map(&mq, q, n_q, n_heads);
-  if (!rc) rc = make_rows_map(&mk, k, n_kv, n_heads);
-  if (!rc) rc = make_rows_map(&mv, v, n_kv, n_heads);
+  int rc = make_rows_map(&mq, q, n_q, n_heads, kAttnQBoxRows);
+  if (!rc) rc = make_rows_map(&mk, k, n_kv, n_heads, kAttnKVBoxRows);
+  if (!rc) rc = make_rows_map(&mv, v, n_kv, n_heads, kAttnKVBoxRows);
   if (rc) return rc;
   return launch_attention_tc(mq, mk, mv, a, 0, n_heads, splits, o, o_part, lse_part, nullptr,
                              (cudaStream_t)stream);

@@ -7,6 +7,10 @@
 namespace sfm {
 
 constexpr int kMaxSplits = 8;
+// TMA box heights of the tcgen05 attention kernel: query and key / value tiles
+// of 128 rows (one 64-dim half of a head per box).
+constexpr int kAttnQBoxRows = 128;
+constexpr int kAttnKVBoxRows = 128;
 
 // Query rows [s * rows_per, (s + 1) * rows_per) of session s attend to key
 // rows [kbase[s], kbase[s] + nkeys[s]) of the layer's K/V arrays.

@@ -37,7 +37,8 @@ using namespace sm100;
 
 namespace atc {
 
-constexpr int BQ = 128, QT = 2, BKV = 128, D = 128;
+constexpr int BQ = kAttnQBoxRows, QT = 2, BKV = kAttnKVBoxRows, D = 128;
+static_assert(BQ == 128 && BKV == 128, "tile shapes fixed by the TMEM / shared-memory plan");
 constexpr int ROWS = BQ * QT;               // query rows per CTA
 constexpr int THREADS = 320;
 constexpr int KST = 3, VST = 2;

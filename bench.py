@@ -115,12 +115,32 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# multi-rank aggregation (one session per rank, no collective on the data path)
+# ---------------------------------------------------------------------------
+def max_over_ranks(ms, device=None):
+    """Largest per-rank device time of the timed region (every rank calls this)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def whole_job_rate(n_units_per_rank, euler_steps, world, ms_max):
+    """Euler denoise steps per second summed over all ranks (weak scaling: each rank
+    solves its own units), timed by the slowest rank."""
+    return euler_steps * n_units_per_rank * world / (ms_max / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # work counts
 # ---------------------------------------------------------------------------
-def flop_counts(w, valid):
+def flop_counts(w, valids):
+    """valids: valid cached tokens of each session of the batch."""
     n, d, hd, f, L = w.n_tokens, w.d_model, w.hd, w.d_mlp, w.n_layers
-    attn = 4 * n * (valid + n) * hd
-    gemm = 2 * n * d * 3 * hd + 2 * n * hd * d + 2 * n * d * f + 2 * n * f * d
+    attn = sum(4 * n * (valid + n) * hd for valid in valids)
+    gemm = len(valids) * (2 * n * d * 3 * hd + 2 * n * hd * d + 2 * n * d * f + 2 * n * f * d)
     return {"attention_per_launch": attn, "gemm_per_layer": gemm,
             "per_euler_step": L * (attn + gemm)}
 
@@ -217,14 +237,31 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def session_caps(w):
+    """Cache capacity (units) of each session the workload runs."""
+    import sfm_synth as S
+    if w.name == S.V02X8.name:
+        return S.session_cache_units(unit_tokens=w.unit_kv_tokens)
+    return [w.cache_units]
+
+
 def config_of(w):
-    return {"workload": f"{w.name} unit: kvcache_append of one {w.unit_kv_tokens}-token slice + "
-                        f"{w.n_steps}-step Euler solve",
-            "tokens_per_unit": w.n_tokens, "video_tokens": w.n_video, "audio_tokens": w.n_audio,
-            "cache_tokens": w.cache_units * w.unit_kv_tokens, "layers": w.n_layers,
-            "d_model": w.d_model, "heads": w.n_heads, "head_dim": w.head_dim, "d_mlp": w.d_mlp,
-            "euler_steps": w.n_steps, "parallelism": "one session per GPU, no collectives",
-            "l2": "inputs larger than L2 (weights + cache read every Euler step)"}
+    caps = session_caps(w)
+    cfg = {"workload": f"{w.name} unit: kvcache_append of one {w.unit_kv_tokens}-token slice + "
+                       f"{w.n_steps}-step Euler solve",
+           "sessions": len(caps), "tokens_per_unit": w.n_tokens, "video_tokens": w.n_video,
+           "audio_tokens": w.n_audio, "layers": w.n_layers,
+           "d_model": w.d_model, "heads": w.n_heads, "head_dim": w.head_dim, "d_mlp": w.d_mlp,
+           "euler_steps": w.n_steps,
+           "l2": "inputs larger than L2 (weights + cache read every Euler step)"}
+    if len(caps) == 1:
+        cfg["cache_tokens"] = caps[0] * w.unit_kv_tokens
+        cfg["parallelism"] = "one session per GPU, no collectives"
+    else:
+        cfg["cache_tokens"] = [c * w.unit_kv_tokens for c in caps]
+        cfg["parallelism"] = (f"{len(caps)} sessions batched per GPU (ragged caches, varlen "
+                              "attention), no collectives")
+    return cfg
 
 
 # ---------------------------------------------------------------------------
@@ -251,26 +288,39 @@ def run_ours(args, w):
             dist.barrier()
 
     weights = S.make_weights(w, device=dev)
-    p = Performer.from_workload(w, weights)
-    s = p.open_session(w.cache_units)
-    k, v = S.make_kv_slices(w, w.cache_units, device=dev)
-    p.kvcache_append(s, k, v)
-    del k, v
+    caps = session_caps(w)
+    n_sess = len(caps)
+    pool = sum(c * w.unit_kv_tokens + w.n_tokens for c in caps)
+    p = Performer.from_workload(w, weights, pool_tokens=pool, max_sessions=n_sess)
+    sessions = []
+    for i, cap in enumerate(caps):
+        s_id = p.open_session(cap)
+        k, v = S.make_kv_slices(w.replace(cache_units=cap), cap, device=dev, seed=S.SEED_CACHE + 10 * i)
+        p.kvcache_append(s_id, k, v)
+        del k, v
+        sessions.append(s_id)
     g = torch.Generator(device=dev)
     g.manual_seed(11 + rank)
     shape = (w.n_layers, w.unit_kv_tokens, w.n_heads, w.head_dim)
     k1 = torch.randn(*shape, generator=g, device=dev).to(torch.bfloat16)
     v1 = torch.randn(*shape, generator=g, device=dev).to(torch.bfloat16)
-    _, eps = S.make_latents(w, device=dev)
-    eps = eps[0].contiguous()
-    z = eps.clone()
+    _, eps = S.make_latents(w, device=dev, n_sessions=n_sess)
+    zs = [eps[i].clone() for i in range(n_sess)]
     taus = S.uniform_taus(w.n_steps)
     torch.cuda.synchronize()
 
+    def solve_all():
+        if n_sess == 1:
+            p.fm_solve(sessions[0], zs[0], taus)
+        else:
+            p.fm_solve_batched(sessions, zs, taus)
+
     def step():
-        p.kvcache_append(s, k1, v1)
-        z.copy_(eps)
-        p.fm_solve(s, z, taus)
+        for s_id in sessions:
+            p.kvcache_append(s_id, k1, v1)
+        for i in range(n_sess):
+            zs[i].copy_(eps[i])
+        solve_all()
 
     for _ in range(args.warmup):
         step()
@@ -293,11 +343,7 @@ def run_ours(args, w):
     prof = L.profile_end()
     launches = L.lib.sfm_kernel_launch_count() - n0
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = t.item()
+    ms_max = max_over_ranks(e0.elapsed_time(e1), dev)
     barrier()
 
     # end to end: host (pinned) inputs copied in and the latents copied out every step
@@ -305,16 +351,20 @@ def run_ours(args, w):
     if not args.no_e2e:
         k1_h = k1.cpu().pin_memory()
         v1_h = v1.cpu().pin_memory()
-        eps_h = eps.cpu().pin_memory()
-        z_h = torch.empty_like(eps_h).pin_memory()
+        eps_h = [eps[i].cpu().pin_memory() for i in range(n_sess)]
+        z_h = [torch.empty_like(e).pin_memory() for e in eps_h]
 
         def e2e_step():
-            k1.copy_(k1_h, non_blocking=True)
-            v1.copy_(v1_h, non_blocking=True)
-            z.copy_(eps_h, non_blocking=True)
-            p.kvcache_append(s, k1, v1)
-            p.fm_solve(s, z, taus)
-            z_h.copy_(z, non_blocking=True)
+            # each session receives its own slice from host memory and returns its latents
+            for s_id in sessions:
+                k1.copy_(k1_h, non_blocking=True)
+                v1.copy_(v1_h, non_blocking=True)
+                p.kvcache_append(s_id, k1, v1)
+            for i in range(n_sess):
+                zs[i].copy_(eps_h[i], non_blocking=True)
+            solve_all()
+            for i in range(n_sess):
+                z_h[i].copy_(zs[i], non_blocking=True)
 
         for _ in range(max(1, args.warmup)):
             e2e_step()
@@ -325,18 +375,15 @@ def run_ours(args, w):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        h2d = k1.numel() * 2 + v1.numel() * 2 + eps.numel() * 4
-        e2e = {"value": w.n_steps * args.steps * world / (te.item() / 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": z.numel() * 4}
+        te_max = max_over_ranks(e0.elapsed_time(e1), dev)
+        h2d = n_sess * (k1.numel() * 2 + v1.numel() * 2 + eps[0].numel() * 4)
+        e2e = {"value": whole_job_rate(args.steps * n_sess, w.n_steps, world, te_max), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": n_sess * eps[0].numel() * 4}
         barrier()
 
     if rank == 0:
         pk = peaks()
-        valid = w.cache_units * w.unit_kv_tokens
-        fl = flop_counts(w, valid)
+        fl = flop_counts(w, [c * w.unit_kv_tokens for c in caps])
         a_ms, a_n = prof["attention"]
         attn_avg_ms = a_ms / max(a_n, 1)
         attn_tflops = fl["attention_per_launch"] / (attn_avg_ms / 1e3) / 1e12
@@ -345,12 +392,12 @@ def run_ours(args, w):
         contraction_flop = args.steps * w.n_steps * fl["per_euler_step"]
         ap_ms, ap_n = prof["append"]
         append_gbs = append_bytes(w) / (ap_ms / max(ap_n, 1) / 1e3) / 1e9 if ap_n else None
+        unit_ms = ms_max / args.steps
         attn_src = os.path.join(ROOT, "streaming_flow_matching_b200", "csrc", "attn_tc.cu")
         traffic = traffic_for(attn_src)
-        unit_ms = ms_max / args.steps
         line = {
             "metric": METRIC,
-            "value": w.n_steps * args.steps * world / (ms_max / 1e3),
+            "value": whole_job_rate(args.steps * n_sess, w.n_steps, world, ms_max),
             "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": unit_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded), resident in HBM",
@@ -374,7 +421,7 @@ def run_ours(args, w):
             "kernel_ms_per_unit": {k2: round(v2[0] / args.steps, 4) for k2, v2 in prof.items()},
             "clocks": clocks,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and n_sess == 1:
             t_step, threads, sample = cpu_sample(w, args.cpu_budget_s)
             line["cpu_baseline"] = {"value": 1.0 / t_step, "unit": UNIT, "cores": threads,
                                     "kind": "oracle", "sample": sample}

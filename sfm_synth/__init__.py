@@ -63,7 +63,10 @@ V01 = Workload("v0.1-192x336", 28, 1536, 12, 128, 6144, 16, 252, 4, 512, 64, 4, 
 # 640x368 unit: 40x23 = 920 video + 4 audio tokens; 48 cached units x 1200 tokens
 V02 = Workload("v0.2-640x368", 28, 3072, 24, 128, 12288, 16, 920, 4, 1200, 48, 4, "bf16")
 
-WORKLOADS = {w.name: w for w in (TINY, V01, V02)}
+# 8 independent sessions at the 640x368 unit shape, ragged caches (see session_cache_units)
+V02X8 = V02.replace(name="v0.2x8-ragged")
+
+WORKLOADS = {w.name: w for w in (TINY, V01, V02, V02X8)}
 
 # isolated attention sweep: cache lengths 4K/16K/64K/128K rounded up to whole 1200-token units
 ATTN_SWEEP_TOKENS = [4800, 16800, 66000, 132000]

@@ -84,8 +84,8 @@ typedef struct sfm_config {
 } sfm_config;
 
 /*
- * Weights of f_theta: device pointers of the config's dtype, borrowed (not
- * copied) for the handle's lifetime.  The per-layer members are HOST arrays
+ * Weights of f_theta: device pointers of the config's dtype, each 16-byte
+ * aligned (else SFM_EINVAL), borrowed (not copied) for the handle's lifetime.  The per-layer members are HOST arrays
  * of n_layers device pointers; the arrays themselves are copied at create.
  *   w_in   [d][C]           x_j = W_in z_j + e_mod[m(j)] + temb(tau)
  *   e_mod  [2][d]           row 0 video, row 1 audio

@@ -53,6 +53,7 @@ struct sfm_handle {
   CUtensorMap map_xn{}, map_ao{}, map_hmlp{};
   CUtensorMap map_q{}, map_kpool{}, map_vpool{};  // attention operands
   std::vector<CUtensorMap> map_wqkv, map_wo, map_w1, map_w2;
+  int bn_qkv = 0, bn_o = 0, bn_up = 0, bn_down = 0;   // N-tile widths the weight maps use
   std::vector<void*> owned;
 
   void* layer_k(int l) const { return (char*)k_pool + (size_t)l * cfg.pool_tokens * hd * es; }
@@ -73,7 +74,7 @@ int validate_config(const sfm_config* c) {
   if (!(c->rms_eps >= 0.0) || !(c->rope_theta > 0.0)) return SFM_EINVAL;
   if (c->max_sessions > kMaxBatch) return SFM_EUNSUPPORTED;
   if ((long long)c->n_layers * c->pool_tokens >= (1LL << 31)) return SFM_EUNSUPPORTED;
-  if (c->c_lat > 64 || c->d_model % 2) return SFM_EUNSUPPORTED;
+  if (c->c_lat > 64 || c->d_model % 2 || c->d_model > 8192) return SFM_EUNSUPPORTED;
   const int hd = c->n_heads * c->head_dim;
   if (c->dtype == SFM_DTYPE_BF16) {
     // GEMM tiles: N in multiples of 128, K in multiples of 64; flash tiles: D_h = 128
@@ -158,7 +159,7 @@ int make_rows_map(CUtensorMap* m, const void* p, long long rows, int heads, int 
   return make_tmap_bf16(m, p, 3, dims, strides, box);
 }
 
-GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err) {
+GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err, int block_n = 0) {
   GemmArgs g{};
   g.M = M;
   g.N = N;
@@ -168,6 +169,7 @@ GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err) {
   g.ldc = ldc;
   g.err = err;
   g.hd = 0;
+  g.block_n = block_n;
   return g;
 }
 
@@ -208,6 +210,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       g.v_layer = (__nv_bfloat16*)h->layer_v(l);
       g.hd = hd;
       g.b = b;
+      g.block_n = h->bn_qkv;
       SFM_TRY(launch_gemm_tc(h->map_xn, h->map_wqkv[l], g, h->sms, s));
     } else {
       {
@@ -230,7 +233,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_O, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_ao, h->map_wo[l],
-                               gemm_args(M, d, hd, EPI_RESID, h->x, d, h->d_err), h->sms, s));
+                               gemm_args(M, d, hd, EPI_RESID, h->x, d, h->d_err, h->bn_o), h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->ao, h->w_o[l], h->x, M, d, hd, EPI_RESID, dt, s));
       }
@@ -243,7 +246,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_UP, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_xn, h->map_w1[l],
-                               gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->d_err), h->sms, s));
+                               gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->d_err, h->bn_up), h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->xn, h->w_1[l], h->hmlp, M, F, d, EPI_GELU, dt, s));
       }
@@ -252,7 +255,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_DOWN, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_hmlp, h->map_w2[l],
-                               gemm_args(M, d, F, EPI_RESID, h->x, d, h->d_err), h->sms, s));
+                               gemm_args(M, d, F, EPI_RESID, h->x, d, h->d_err, h->bn_down), h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->hmlp, h->w_2[l], h->x, M, d, F, EPI_RESID, dt, s));
       }
@@ -312,7 +315,9 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
   }
   if (w) {
     const void* const* arrays[6] = {w->g_attn, w->w_qkv, w->w_o, w->g_mlp, w->w_1, w->w_2};
-    if (!w->w_in || !w->e_mod || !w->g_final || !w->w_out) rc = SFM_EINVAL;
+    if (!aligned16(w->w_in) || !aligned16(w->e_mod) || !aligned16(w->g_final) ||
+        !aligned16(w->w_out) || !w->w_in || !w->e_mod || !w->g_final || !w->w_out)
+      rc = SFM_EINVAL;
     for (int a = 0; a < 6 && !rc; ++a) {
       if (!arrays[a]) rc = SFM_EINVAL;
       for (int l = 0; l < cfg->n_layers && !rc; ++l)
@@ -391,11 +396,17 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     h->map_wo.resize(L_);
     h->map_w1.resize(L_);
     h->map_w2.resize(L_);
+    // tile widths chosen for a full batch (max_sessions units)
+    h->bn_qkv = gemm_tc_block_n((int)M, 3 * hd_, hd_, EPI_QKV, h->sms);
+    h->bn_o = gemm_tc_block_n((int)M, d_, 0, EPI_RESID, h->sms);
+    h->bn_up = gemm_tc_block_n((int)M, F_, 0, EPI_GELU, h->sms);
+    h->bn_down = gemm_tc_block_n((int)M, d_, 0, EPI_RESID, h->sms);
+    if (!h->bn_qkv || !h->bn_o || !h->bn_up || !h->bn_down) rc = SFM_EUNSUPPORTED;
     for (int l = 0; l < L_ && !rc; ++l) {
-      rc = make_b_map(&h->map_wqkv[l], h->w_qkv[l], 3 * hd_, d_, gemm_tc_block_n(3 * hd_, hd_, EPI_QKV));
-      if (!rc) rc = make_b_map(&h->map_wo[l], h->w_o[l], d_, hd_, gemm_tc_block_n(d_, 0, EPI_RESID));
-      if (!rc) rc = make_b_map(&h->map_w1[l], h->w_1[l], F_, d_, gemm_tc_block_n(F_, 0, EPI_GELU));
-      if (!rc) rc = make_b_map(&h->map_w2[l], h->w_2[l], d_, F_, gemm_tc_block_n(d_, 0, EPI_RESID));
+      rc = make_b_map(&h->map_wqkv[l], h->w_qkv[l], 3 * hd_, d_, h->bn_qkv);
+      if (!rc) rc = make_b_map(&h->map_wo[l], h->w_o[l], d_, hd_, h->bn_o);
+      if (!rc) rc = make_b_map(&h->map_w1[l], h->w_1[l], F_, d_, h->bn_up);
+      if (!rc) rc = make_b_map(&h->map_w2[l], h->w_2[l], d_, F_, h->bn_down);
     }
   }
   if (rc) {
@@ -620,15 +631,16 @@ int sfm_linear(const void* x, const void* w, void* y, int M, int N, int K, int e
   }
   if (dtype != SFM_DTYPE_BF16) return SFM_EINVAL;
   if (N % 128 || K % 64) return SFM_EUNSUPPORTED;
-  const int bn = gemm_tc_block_n(N, 0, epi);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int bn = gemm_tc_block_n(M, N, 0, epi, sms);
+  if (!bn) return SFM_EUNSUPPORTED;
   CUtensorMap ma, mb;
   int rc = make_a_map(&ma, x, M, K);
   if (!rc) rc = make_b_map(&mb, w, N, K, bn);
   if (rc) return rc;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return launch_gemm_tc(ma, mb, gemm_args(M, N, K, epi, y, N, nullptr), sms, (cudaStream_t)stream);
+  return launch_gemm_tc(ma, mb, gemm_args(M, N, K, epi, y, N, nullptr, bn), sms, (cudaStream_t)stream);
 }
 
 const char* sfm_strerror(int status) {

@@ -29,8 +29,8 @@ int launch_attention(const AttnDesc& a, const void* q, const void* k, const void
 int launch_attention_merge(const float* o_part, const float* lse_part, void* o,
                            long long total_rows, int n_heads, int n_splits, cudaStream_t s);
 
-// tcgen05 attention (bf16, D = 128).  Split count for a batch; the SM count is
-// an input so the choice is reproducible (the standalone call assumes 148).
+// tcgen05 attention (bf16, D = 128).  Split count for a batch; the SM count is an input so the choice is
+// reproducible (the standalone call assumes 148).
 int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads,
                         int sms);
 // mq: map over the query rows [rows][H][128]; mk, mv: maps over the key rows, of

@@ -302,11 +302,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (c + 1 < 4) tmem_ld32(tmem + lane_base + col_s + (c + 1) * 32, u[(c + 1) & 1]);
           const float* sv = reinterpret_cast<const float*>(u[c & 1]);
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            m4[0] = fmaxf(m4[0], sv[i]);
-            m4[1] = fmaxf(m4[1], sv[i + 1]);
-            m4[2] = fmaxf(m4[2], sv[i + 2]);
-            m4[3] = fmaxf(m4[3], sv[i + 3]);
+          for (int i = 0; i < 32; i += 8) {
+            m4[0] = fmax3(m4[0], sv[i], sv[i + 1]);
+            m4[1] = fmax3(m4[1], sv[i + 2], sv[i + 3]);
+            m4[2] = fmax3(m4[2], sv[i + 4], sv[i + 5]);
+            m4[3] = fmax3(m4[3], sv[i + 6], sv[i + 7]);
           }
           if (c + 1 < 4) tmem_wait_ld(u[(c + 1) & 1]);
         }

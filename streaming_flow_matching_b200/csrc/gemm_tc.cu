@@ -27,11 +27,12 @@ constexpr int BM = 128, BK = 64;
 constexpr int THREADS = 192;
 
 template <int BN> struct Cfg {
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 192 ? 5 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int ACC_COLS = BN == 128 ? 128 : 256;     // TMEM columns between the two accumulators
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
 };
 
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        const uint32_t d = tmem + (uint32_t)(acc * C::ACC_COLS);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&full[s], ph, abort, args.err, 0x103)) {
             ok = false;
@@ -188,7 +189,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_ph, abort, args.err, 0x104))) break;
       tc_fence_after();
       const int row = m0 + quarter * 32 + lane;
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
       if (EPI == EPI_QKV) {
         const int hd = args.hd;
         const int section = n0 / hd;           // 0 q, 1 k, 2 v (a tile never straddles)
@@ -295,16 +296,31 @@ int launch_bn(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, 
 
 }  // namespace gtc
 
-int gemm_tc_block_n(int N, int hd, int epi) {
-  if (epi == EPI_QKV) return (hd % 256 == 0) ? 256 : 128;
-  return (N % 256 == 0) ? 256 : 128;
+int gemm_tc_block_n(int M, int N, int hd, int epi, int sms) {
+  // N-tile width minimising (waves of the persistent grid) x (work per tile);
+  // ties go to the wider tile.  The QKV epilogue works on whole 128-wide heads.
+  const int cands[3] = {256, 192, 128};
+  const long long m_tiles = (M + gtc::BM - 1) / gtc::BM;
+  int best = 0;
+  long long best_cost = 0;
+  for (int bn : cands) {
+    if (N % bn) continue;
+    if (epi == EPI_QKV && (bn % 128 || hd % bn)) continue;
+    const long long tiles = m_tiles * (N / bn);
+    const long long cost = ((tiles + sms - 1) / sms) * bn;
+    if (!best || cost < best_cost) {
+      best = bn;
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
 int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,
                    cudaStream_t s) {
   if (args.M <= 0) return SFM_OK;
-  const int bn = gemm_tc_block_n(args.N, args.hd, args.epi);
-  if (args.N % bn || args.K % gtc::BK || args.K <= 0) return SFM_EUNSUPPORTED;
+  const int bn = args.block_n ? args.block_n : gemm_tc_block_n(args.M, args.N, args.hd, args.epi, sms);
+  if (!bn || args.N % bn || args.K % gtc::BK || args.K <= 0) return SFM_EUNSUPPORTED;
   if (args.epi == EPI_QKV && (args.hd % bn || args.N != 3 * args.hd)) return SFM_EUNSUPPORTED;
 #define SFM_GTC(BN_, E)                                          \
   if (bn == BN_ && args.epi == E) return gtc::launch_bn<BN_, E>(a, b, args, sms, s);
@@ -313,6 +329,10 @@ int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& a
   SFM_GTC(256, EPI_RESID)
   SFM_GTC(256, EPI_STORE)
   SFM_GTC(256, EPI_QKV)
+  SFM_GTC(192, EPI_F32)
+  SFM_GTC(192, EPI_GELU)
+  SFM_GTC(192, EPI_RESID)
+  SFM_GTC(192, EPI_STORE)
   SFM_GTC(128, EPI_F32)
   SFM_GTC(128, EPI_GELU)
   SFM_GTC(128, EPI_RESID)

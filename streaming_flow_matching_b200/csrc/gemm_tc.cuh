@@ -20,10 +20,11 @@ struct GemmArgs {
   __nv_bfloat16* v_layer;
   int hd;
   BatchDesc b;
+  int block_n;           // N-tile width the B tensor map was built for (0: choose)
 };
 
-// Block N the kernel uses for a problem (128 or 256).
-int gemm_tc_block_n(int N, int hd, int epi);
+// N-tile width (256, 192 or 128) for an M x N problem on `sms` SMs; 0 if none fits.
+int gemm_tc_block_n(int M, int N, int hd, int epi, int sms);
 // A: tensor map over [M_alloc][K] bf16, box {64, 128}; B: over [N][K], box {64, block_n}.
 int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,
                    cudaStream_t s);

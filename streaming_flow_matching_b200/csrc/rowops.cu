@@ -37,8 +37,11 @@ __device__ __forceinline__ float warp_sum(float v) {
 // ---------------------------------------------------------------------------
 constexpr int kEmbedRows = 32;
 
-template <typename T>
-__global__ void embed_kernel(BatchDesc b, PtrTable z, const T* __restrict__ w_in,
+// CL: compile-time bound on c_lat (16, or 64 for any c_lat <= 64), so the
+// W_in row stays in registers.
+template <typename T, int CL>
+__global__ void embed_kernel(const __grid_constant__ BatchDesc b, const __grid_constant__ PtrTable z,
+                             const T* __restrict__ w_in,
                              const T* __restrict__ e_mod, float tau, float* __restrict__ x, int d,
                              int c_lat) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -48,9 +51,9 @@ __global__ void embed_kernel(BatchDesc b, PtrTable z, const T* __restrict__ w_in
   const double w = pow(10000.0, -2.0 * (double)ii / (double)d);
   const double ang = 1000.0 * (double)tau * w;
   const float te = (float)(i < half ? sin(ang) : cos(ang));
-  float wr[64];
-#pragma unroll 16
-  for (int c = 0; c < c_lat; ++c) wr[c] = to_f(w_in[(size_t)i * c_lat + c]);
+  float wr[CL];
+#pragma unroll
+  for (int c = 0; c < CL; ++c) wr[c] = c < c_lat ? to_f(w_in[(size_t)i * c_lat + c]) : 0.f;
   const float em_v = to_f(e_mod[i]);
   const float em_a = to_f(e_mod[d + i]);
   const int rows = b.n * b.n_tok;
@@ -60,8 +63,9 @@ __global__ void embed_kernel(BatchDesc b, PtrTable z, const T* __restrict__ w_in
     const int j = r - sess * b.n_tok;
     const float* zr = z.p[sess] + (size_t)j * c_lat;
     float acc = 0.f;
-#pragma unroll 16
-    for (int c = 0; c < c_lat; ++c) acc = fmaf(zr[c], wr[c], acc);
+#pragma unroll
+    for (int c = 0; c < CL; ++c)
+      if (c < c_lat) acc = fmaf(zr[c], wr[c], acc);
     x[(size_t)r * d + i] = acc + (j < b.n_video ? em_v : em_a) + te;
   }
 }
@@ -72,54 +76,97 @@ int launch_embed(const BatchDesc& b, float* const* z, const void* w_in, const vo
   for (int i = 0; i < b.n; ++i) t.p[i] = z[i];
   const int rows = b.n * b.n_tok;
   dim3 grid((d + 127) / 128, (rows + kEmbedRows - 1) / kEmbedRows);
-  if (dtype == SFM_DTYPE_BF16)
-    embed_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(b, t, (const __nv_bfloat16*)w_in,
-                                                     (const __nv_bfloat16*)e_mod, tau, x, d, c_lat);
-  else
-    embed_kernel<float><<<grid, 128, 0, s>>>(b, t, (const float*)w_in, (const float*)e_mod, tau,
-                                             x, d, c_lat);
+  if (c_lat > 64) return SFM_EUNSUPPORTED;
+  const bool c16 = c_lat == 16;
+  if (dtype == SFM_DTYPE_BF16) {
+    auto k = c16 ? embed_kernel<__nv_bfloat16, 16> : embed_kernel<__nv_bfloat16, 64>;
+    k<<<grid, 128, 0, s>>>(b, t, (const __nv_bfloat16*)w_in, (const __nv_bfloat16*)e_mod, tau, x,
+                           d, c_lat);
+  } else {
+    auto k = c16 ? embed_kernel<float, 16> : embed_kernel<float, 64>;
+    k<<<grid, 128, 0, s>>>(b, t, (const float*)w_in, (const float*)e_mod, tau, x, d, c_lat);
+  }
   return record_cuda(cudaGetLastError());
 }
 
 // ---------------------------------------------------------------------------
-// RMSNorm: one warp per row, float4 loads.
+// RMSNorm: one CTA per row; each thread holds 8 consecutive elements in
+// registers (one read of x), block reduction of the sum of squares, 16-byte
+// stores of the bf16 (or 2 x 16-byte fp32) output.  d / 8 <= 1024.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void store8(__nv_bfloat16* o, const float* v) {
+  uint4 u;
+  __nv_bfloat162 t;
+  t = __floats2bfloat162_rn(v[0], v[1]); u.x = *reinterpret_cast<uint32_t*>(&t);
+  t = __floats2bfloat162_rn(v[2], v[3]); u.y = *reinterpret_cast<uint32_t*>(&t);
+  t = __floats2bfloat162_rn(v[4], v[5]); u.z = *reinterpret_cast<uint32_t*>(&t);
+  t = __floats2bfloat162_rn(v[6], v[7]); u.w = *reinterpret_cast<uint32_t*>(&t);
+  *reinterpret_cast<uint4*>(o) = u;
+}
+__device__ __forceinline__ void store8(float* o, const float* v) {
+  reinterpret_cast<float4*>(o)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(o)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float* v) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float* v) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 template <typename T>
-__global__ void rmsnorm_kernel(const float* __restrict__ x, const T* __restrict__ g,
-                               T* __restrict__ out, int rows, int d, float eps) {
-  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * d);
-  const int nv = d / 4;
+__global__ void __launch_bounds__(1024) rmsnorm_kernel(const float* __restrict__ x,
+                                                      const T* __restrict__ g,
+                                                      T* __restrict__ out, int d, float eps) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  const int c = threadIdx.x * 8;
+  const bool on = c < d;
+  float v[8];
   float ss = 0.f;
-  for (int c = lane; c < nv; c += 32) {
-    const float4 a = xr[c];
-    ss = fmaf(a.x, a.x, ss);
-    ss = fmaf(a.y, a.y, ss);
-    ss = fmaf(a.z, a.z, ss);
-    ss = fmaf(a.w, a.w, ss);
+  if (on) {
+    load8(x + (size_t)row * d + c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss = fmaf(v[i], v[i], ss);
   }
   ss = warp_sum(ss);
-  const float r = rsqrtf(ss / (float)d + eps);
-  T* o = out + (size_t)row * d;
-  for (int c = lane; c < nv; c += 32) {
-    const float4 a = xr[c];
-    o[4 * c + 0] = from_f<T>(a.x * r * to_f(g[4 * c + 0]));
-    o[4 * c + 1] = from_f<T>(a.y * r * to_f(g[4 * c + 1]));
-    o[4 * c + 2] = from_f<T>(a.z * r * to_f(g[4 * c + 2]));
-    o[4 * c + 3] = from_f<T>(a.w * r * to_f(g[4 * c + 3]));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  if (warp == 0) {
+    float t = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.f;
+    t = warp_sum(t);
+    if (lane == 0) red[0] = t;
   }
+  __syncthreads();
+  if (!on) return;
+  const float r = rsqrtf(red[0] / (float)d + eps);
+  float gv[8];
+  load8(g + c, gv);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = v[i] * r * gv[i];
+  store8(out + (size_t)row * d + c, v);
 }
 
 int launch_rmsnorm(const float* x, const void* g, void* out, int rows, int d, float eps,
                    int dtype, cudaStream_t s) {
-  const int blocks = (rows + 7) / 8;
+  if (rows <= 0) return SFM_OK;
+  if (d % 8 || d / 8 > 1024) return SFM_EUNSUPPORTED;
+  const int threads = ((d / 8) + 31) / 32 * 32;
   if (dtype == SFM_DTYPE_BF16)
-    rmsnorm_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(x, (const __nv_bfloat16*)g,
-                                                         (__nv_bfloat16*)out, rows, d, eps);
+    rmsnorm_kernel<__nv_bfloat16><<<rows, threads, 0, s>>>(x, (const __nv_bfloat16*)g,
+                                                          (__nv_bfloat16*)out, d, eps);
   else
-    rmsnorm_kernel<float><<<blocks, 256, 0, s>>>(x, (const float*)g, (float*)out, rows, d, eps);
+    rmsnorm_kernel<float><<<rows, threads, 0, s>>>(x, (const float*)g, (float*)out, d, eps);
   return record_cuda(cudaGetLastError());
 }
 
@@ -206,46 +253,124 @@ int launch_rope_scatter(const BatchDesc& b, const float* qkv, const float* cos_t
 }
 
 // ---------------------------------------------------------------------------
-// Velocity head fused with the Euler update: one warp per token row.
+// Velocity head fused with the final RMSNorm and the Euler update.  One CTA of
+// kHeadThreads per kHeadRows token rows: every thread walks a strided set of
+// 4-column groups, accumulating sum(x^2) per row and x*g*W_out for 16 output
+// channels per row, so the RMS scale is applied once to the finished dot
+// products.  The 64 partial sums per thread are reduced across the warp by
+// halving exchanges (each step hands half of the values to the partner lane),
+// which leaves 2 totals per lane after 62 shuffles; warps then combine
+// through shared memory.
 // ---------------------------------------------------------------------------
+constexpr int kHeadRows = 4, kHeadThreads = 256, kHeadCh = 16;
+constexpr int kHeadVals = kHeadRows * kHeadCh;   // 64 accumulators per thread
+
+__device__ __forceinline__ void load4(const float* p, float* o) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float* o) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+  o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+}
+
+template <int N>
+__device__ __forceinline__ void halve_step(float* acc, int lane, int o) {
+  const bool up = (lane & o) != 0;
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const float send = up ? acc[j] : acc[j + N];
+    const float keep = up ? acc[j + N] : acc[j];
+    acc[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+  }
+}
+
 template <typename T>
-__global__ void head_euler_kernel(BatchDesc b, const float* __restrict__ x,
-                                  const T* __restrict__ g, const T* __restrict__ w_out,
-                                  PtrTable z, PtrTable v_out, float dtau, int d, int c_lat,
-                                  float eps) {
-  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(kHeadThreads)
+    head_euler_kernel(const __grid_constant__ BatchDesc b, const float* __restrict__ x, const T* __restrict__ g,
+                      const T* __restrict__ w_out, const __grid_constant__ PtrTable z,
+                      const __grid_constant__ PtrTable v_out, float dtau, int d,
+                      int c_lat, float eps) {
+  __shared__ float red[kHeadThreads / 32][kHeadVals];
+  __shared__ float red_ss[kHeadThreads / 32][kHeadRows];
   const int rows = b.n * b.n_tok;
-  if (row >= rows) return;
-  const int sess = row / b.n_tok;
-  const int j = row - sess * b.n_tok;
-  const float* xr = x + (size_t)row * d;
-  float ss = 0.f;
-  for (int i = lane; i < d; i += 32) ss = fmaf(xr[i], xr[i], ss);
-  ss = warp_sum(ss);
-  const float rinv = rsqrtf(ss / (float)d + eps);
-  for (int c0 = 0; c0 < c_lat; c0 += 16) {
-    float acc[16];
+  const int row0 = blockIdx.x * kHeadRows;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nr = rows - row0 < kHeadRows ? rows - row0 : kHeadRows;
+  for (int c0 = 0; c0 < c_lat; c0 += kHeadCh) {
+    const int nc = c_lat - c0 < kHeadCh ? c_lat - c0 : kHeadCh;
+    float acc[kHeadVals];
+    float ss[kHeadRows];
 #pragma unroll
-    for (int c = 0; c < 16; ++c) acc[c] = 0.f;
-    for (int i = lane; i < d; i += 32) {
-      const float xn = xr[i] * rinv * to_f(g[i]);
+    for (int k = 0; k < kHeadVals; ++k) acc[k] = 0.f;
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        if (c0 + c < c_lat) acc[c] = fmaf(xn, to_f(w_out[(size_t)(c0 + c) * d + i]), acc[c]);
+    for (int q = 0; q < kHeadRows; ++q) ss[q] = 0.f;
+    for (int i = 4 * threadIdx.x; i < d; i += 4 * kHeadThreads) {
+      float gi[4], xv[kHeadRows][4];
+      load4(g + i, gi);
+#pragma unroll
+      for (int q = 0; q < kHeadRows; ++q) {
+        if (q < nr) {
+          load4(x + (size_t)(row0 + q) * d + i, xv[q]);
+        } else {
+          xv[q][0] = xv[q][1] = xv[q][2] = xv[q][3] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          ss[q] = fmaf(xv[q][e], xv[q][e], ss[q]);
+          xv[q][e] *= gi[e];
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < kHeadCh; ++c) {
+        float wv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (c < nc) load4(w_out + (size_t)(c0 + c) * d + i, wv);
+#pragma unroll
+        for (int q = 0; q < kHeadRows; ++q)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[q * kHeadCh + c] = fmaf(xv[q][e], wv[e], acc[q * kHeadCh + c]);
+      }
     }
+    // halving exchange: after the step with offset o a lane keeps the half of
+    // its values selected by (lane & o); lane L ends holding totals 2L, 2L+1
+    halve_step<32>(acc, lane, 16);
+    halve_step<16>(acc, lane, 8);
+    halve_step<8>(acc, lane, 4);
+    halve_step<4>(acc, lane, 2);
+    halve_step<2>(acc, lane, 1);
 #pragma unroll
-    for (int c = 0; c < 16; ++c) acc[c] = warp_sum(acc[c]);
-    float mine = 0.f;
+    for (int q = 0; q < kHeadRows; ++q) ss[q] = warp_sum(ss[q]);
+    red[warp][2 * lane] = acc[0];
+    red[warp][2 * lane + 1] = acc[1];
+    if (lane < kHeadRows) {
+      float mine = ss[0];
 #pragma unroll
-    for (int c = 0; c < 16; ++c)
-      if (lane == c) mine = acc[c];
-    const int ch = c0 + lane;
-    if (lane < 16 && ch < c_lat) {
-      float* zr = z.p[sess] + (size_t)j * c_lat;
-      zr[ch] = fmaf(dtau, mine, zr[ch]);
-      if (v_out.p[sess]) v_out.p[sess][(size_t)j * c_lat + ch] = mine;
+      for (int q = 1; q < kHeadRows; ++q)
+        if (lane == q) mine = ss[q];
+      red_ss[warp][lane] = mine;
     }
+    __syncthreads();
+    if (threadIdx.x < kHeadVals) {
+      const int q = threadIdx.x / kHeadCh, c = threadIdx.x % kHeadCh;
+      float dot = 0.f, sq = 0.f;
+#pragma unroll
+      for (int w = 0; w < kHeadThreads / 32; ++w) {
+        dot += red[w][threadIdx.x];
+        sq += red_ss[w][q];
+      }
+      const int row = row0 + q;
+      if (q < nr && c < nc) {
+        const float v = dot * rsqrtf(sq / (float)d + eps);
+        const int sess = row / b.n_tok;
+        const int j = row - sess * b.n_tok;
+        float* zr = z.p[sess] + (size_t)j * c_lat + c0 + c;
+        *zr = fmaf(dtau, v, *zr);
+        if (v_out.p[sess]) v_out.p[sess][(size_t)j * c_lat + c0 + c] = v;
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -258,12 +383,15 @@ int launch_head_euler(const BatchDesc& b, const float* x, const void* g, const v
     vt.p[i] = v_out ? v_out[i] : nullptr;
   }
   const int rows = b.n * b.n_tok;
-  const int blocks = (rows + 7) / 8;
+  const int blocks = (rows + kHeadRows - 1) / kHeadRows;
+  if (blocks == 0) return SFM_OK;
+  if (d % 4 || ((uintptr_t)g & 15u) || ((uintptr_t)w_out & 15u) || ((uintptr_t)x & 15u))
+    return SFM_EUNSUPPORTED;
   if (dtype == SFM_DTYPE_BF16)
-    head_euler_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+    head_euler_kernel<__nv_bfloat16><<<blocks, kHeadThreads, 0, s>>>(
         b, x, (const __nv_bfloat16*)g, (const __nv_bfloat16*)w_out, zt, vt, dtau, d, c_lat, eps);
   else
-    head_euler_kernel<float><<<blocks, 256, 0, s>>>(b, x, (const float*)g, (const float*)w_out,
+    head_euler_kernel<float><<<blocks, kHeadThreads, 0, s>>>(b, x, (const float*)g, (const float*)w_out,
                                                     zt, vt, dtau, d, c_lat, eps);
   return record_cuda(cudaGetLastError());
 }

@@ -1,6 +1,7 @@
 """Dense projections through the C ABI (sfm_linear) against the oracle's
-matmul in fp64: tcgen05 tiles with ragged M tails, both N-tile widths, every
-epilogue; fp32 mode on the CUDA cores."""
+matmul in fp64: tcgen05 tiles with ragged M tails, every N-tile width (128,
+192, 256: the width follows from M and N), every epilogue; fp32 mode on the
+CUDA cores."""
 import numpy as np
 import pytest
 import torch
@@ -35,7 +36,8 @@ def test_linear_bf16_f32_out(cuda_device, M, N, K):
     assert e <= 5e-5, e
 
 
-@pytest.mark.parametrize("M,N,K", [(130, 256, 128), (300, 384, 192), (924, 12288, 3072)])
+@pytest.mark.parametrize("M,N,K", [(130, 256, 128), (300, 384, 192), (924, 3072, 3072),
+                                   (924, 12288, 3072)])
 def test_linear_bf16_epilogues(cuda_device, M, N, K):
     from streaming_flow_matching_b200 import linear
     x, w = _inputs(M, N, K, torch.bfloat16, 7 * M + N)

@@ -130,7 +130,10 @@ def test_v02_width_full_cache_step_matches_oracle(cuda_device):
 # attention
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("n_q,n_kv", [(1, 1), (17, 5), (64, 64), (204, 704), (924, 5724)])
+# up to 256 query rows run on single CTAs, more on CTA pairs (512 rows per pair):
+# 257 leaves the second CTA of the pair without rows, 513 a pair with one row
+@pytest.mark.parametrize("n_q,n_kv", [(1, 1), (17, 5), (64, 64), (204, 704), (924, 5724),
+                                      (257, 1), (300, 129), (513, 1000), (1030, 3000)])
 def test_attention_bf16_matches_oracle(cuda_device, n_q, n_kv):
     from streaming_flow_matching_b200 import attention
     q, k, v = S.make_qkv(n_q, n_kv, 3, 128)
@@ -156,19 +159,21 @@ def test_attention_sweep_sampled_rows(cuda_device, n_kv):
     assert e <= BF16_TOL, e
 
 
+@pytest.mark.parametrize("n_q", [128, 640])
 @pytest.mark.parametrize("n_kv", [512, 20000])
-def test_attention_max_jump_in_some_rows_only(cuda_device, n_kv):
+def test_attention_max_jump_in_some_rows_only(cuda_device, n_q, n_kv):
     # A few rows (one lane in each of several warps) meet a key aligned with their
     # query in a later key tile: their running max jumps by far more than 2^8 while
     # the rest of the warp's rows do not, so the online-softmax rescale of O is
     # needed by only some rows of a warp.
     from streaming_flow_matching_b200 import attention
     g = torch.Generator().manual_seed(21)
-    n_q, H = 128, 2
+    H = 2
     q = torch.randn(n_q, H, 128, generator=g)
     k = 0.1 * torch.randn(n_kv, H, 128, generator=g)
     v = torch.randn(n_kv, H, 128, generator=g)
-    for i, r in enumerate([3, 40, 77, 101]):
+    rows = [3, 40, 77, 101] + ([300, 333, 600] if n_q > 128 else [])
+    for i, r in enumerate(rows):
         k[300 + i] = 2.0 * q[r]
     q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
     o = attention(q.cuda(), k.cuda(), v.cuda())

@@ -16,12 +16,13 @@
 //               S_t of the next key tile is issued once O_t's P V has completed
 //               (P_t aliases S_t in TMEM).
 //   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B (thread = query
-//               row): two passes over the S row in TMEM (row max, then
-//               p = 2^(s scale - m)), P written back to TMEM as packed bf16;
-//               O rescaled in TMEM only when a row's running max grows by more
-//               than 2^8 (decided per warp: the TMEM accesses are collective);
-//               final O / l written as bf16 (one split) or as fp32 partials +
-//               log2-sum-exp (several splits).
+//               row): one pass over the S row in TMEM computes
+//               p = 2^(s scale - m) against the running max m together with the
+//               tile's max; P is held in registers and written back over S as
+//               packed bf16.  Only when a row's max grows by more than 2^8
+//               (decided per warp: the TMEM accesses are collective) is O
+//               rescaled in TMEM and P recomputed from S.  Final O / l written
+//               as bf16 (one split) or as fp32 partials + log2-sum-exp.
 // TMEM columns: tile A S/P [0,128) O [128,256); tile B S/P [256,384) O [384,512).
 // The last, partial key tile is masked in S, and its V rows past the key range
 // are zeroed in shared memory before P V, so rows outside the range never
@@ -113,7 +114,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int t = 0; t < QT; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&p_full[t], 4);          // one arrival per softmax warp of the tile
       mbar_init(&o_done[t], 1);
     }
     mbar_init(drain, 1);
@@ -290,10 +291,58 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tmem_st_wait();
       }
-      // pass 1: row max of the raw logits (the scale is positive); the load of the
-      // next 32-column chunk overlaps the max over the current one
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      {
+      // P = 2^(s scale - m) with m the running row max.  From the second key tile on, one
+      // pass over the S row computes P against the running max and the tile's max
+      // together; only when some row of the warp grows by more than 2^8 is that
+      // attempt dropped: O is rescaled and P recomputed from S (still intact in TMEM,
+      // as P is held in registers until the row is done).  The first tile takes its
+      // max first.  Loads of the next 32-column chunk overlap work on the current one.
+      uint32_t pk[4][16];
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      float mx = -INFINITY;
+      bool fresh = j == 0;                                // P still to be computed
+      if (!fresh) {
+        const float neg_m = -m;
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        uint32_t u[2][32];
+        tmem_ld32(tmem + lane_base + col_s, u[0]);
+        tmem_wait_ld(u[0]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c + 1 < 4) tmem_ld32(tmem + lane_base + col_s + (c + 1) * 32, u[(c + 1) & 1]);
+          const float* sv = reinterpret_cast<const float*>(u[c & 1]);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            m4[i & 3] = fmax3(m4[i & 3], sv[2 * i], sv[2 * i + 1]);
+            const float p0 = ex2_approx(fmaf(sv[2 * i], sc, neg_m));
+            const float p1 = ex2_approx(fmaf(sv[2 * i + 1], sc, neg_m));
+            l4[(2 * i) & 3] += p0;
+            l4[(2 * i + 1) & 3] += p1;
+            pk[c][i] = pack_bf16x2(p0, p1);
+          }
+          if (c + 1 < 4) tmem_wait_ld(u[(c + 1) & 1]);
+        }
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
+        if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+          // O_t's previous P V has completed (S_t(j) was issued after it): rescale it
+          const float m_new = fmaxf(m, mx);
+          const float alpha = ex2_approx(m - m_new);
+          l *= alpha;
+          m = m_new;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_base + col_o + c * 32, o);
+            tmem_wait_ld(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tmem + lane_base + col_o + c * 32, o);
+          }
+          fresh = true;
+        }
+      } else {
+        // first tile: row max of the raw logits (the scale is positive)
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         uint32_t u[2][32];
         tmem_ld32(tmem + lane_base + col_s, u[0]);
         tmem_wait_ld(u[0]);
@@ -310,32 +359,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           if (c + 1 < 4) tmem_wait_ld(u[(c + 1) & 1]);
         }
+        m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
       }
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
-      // O_t's previous P V has completed (S_t(j) was issued after it), so O_t may be rescaled
-      if (j == 0) {
-        m = mx;
-      } else if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
-        const float m_new = fmaxf(m, mx);
-        const float alpha = ex2_approx(m - m_new);
-        l *= alpha;
-        m = m_new;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + col_o + c * 32, o);
-          tmem_wait_ld(o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + lane_base + col_o + c * 32, o);
-        }
-      }
-      // pass 2: p = 2^(s scale - m) as packed bf16 pairs written over the S row:
-      // keys [32 c, 32 c + 32) -> P columns [16 c, 16 c + 16), which hold S columns
-      // already read (chunk c itself or chunk c - 1); the next chunk's load overlaps
-      const float neg_m = -m;
-      float l4[4] = {0.f, 0.f, 0.f, 0.f};
-      {
+      if (__any_sync(0xffffffffu, fresh)) {
+        const float neg_m = -m;
+        l4[0] = l4[1] = l4[2] = l4[3] = 0.f;
         uint32_t u[2][32];
         tmem_ld32(tmem + lane_base + col_s, u[0]);
         tmem_wait_ld(u[0]);
@@ -343,19 +371,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < 4; ++c) {
           if (c + 1 < 4) tmem_ld32(tmem + lane_base + col_s + (c + 1) * 32, u[(c + 1) & 1]);
           const float* sv = reinterpret_cast<const float*>(u[c & 1]);
-          uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float p0 = ex2_approx(fmaf(sv[2 * i], sc, neg_m));
             const float p1 = ex2_approx(fmaf(sv[2 * i + 1], sc, neg_m));
             l4[(2 * i) & 3] += p0;
             l4[(2 * i + 1) & 3] += p1;
-            pk[i] = pack_bf16x2(p0, p1);
+            pk[c][i] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(tmem + lane_base + col_s + c * 16, pk);
           if (c + 1 < 4) tmem_wait_ld(u[(c + 1) & 1]);
         }
       }
+      // P as packed bf16 pairs over the S row: keys [32 c, 32 c + 32) -> columns [16 c, 16 c + 16)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_st16(tmem + lane_base + col_s + c * 16, pk[c]);
       l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       tmem_st_wait();
       if (t == 0 && kvalid < BKV) {
@@ -379,7 +408,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         fence_proxy_async_smem();
       }
       tc_fence_before();
-      mbar_arrive(&p_full[t]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
     // ---- output ----
     if (ok && T > 0) {

@@ -186,9 +186,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t acc_ph = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
       const int m0 = (t % m_tiles) * BM, n0 = (t / m_tiles) * BN;
+      const int row = m0 + quarter * 32 + lane;
+      const bool live = row < args.M;
+      // residual add: this row's fp32 slice of chunk 0 is loaded (from L2) while the
+      // tile's MMAs finish; chunk c + 1 while chunk c is read from TMEM and stored
+      float4 res[2][8];
+      if (EPI == EPI_RESID && live) {
+        const float4* src = reinterpret_cast<const float4*>((const float*)args.C + (size_t)row * args.ldc + n0);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) res[0][q] = src[q];
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_ph, abort, args.err, 0x104))) break;
       tc_fence_after();
-      const int row = m0 + quarter * 32 + lane;
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
       if (EPI == EPI_QKV) {
         const int hd = args.hd;
@@ -204,14 +213,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (row >= args.M) continue;
             float a[32], b[32];
             if (section < 2) {
-              const float* cs = args.cos_t + (size_t)row * 64 + half * 32;
-              const float* sn = args.sin_t + (size_t)row * 64 + half * 32;
+              // this row's cos / sin for pairs [32 half, 32 half + 32): 16-byte loads
+              const float4* cs = reinterpret_cast<const float4*>(args.cos_t + (size_t)row * 64 + half * 32);
+              const float4* sn = reinterpret_cast<const float4*>(args.sin_t + (size_t)row * 64 + half * 32);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float x = __uint_as_float(ra[i]), y = __uint_as_float(rb[i]);
-                const float c = cs[i], s = sn[i];
-                a[i] = x * c - y * s;
-                b[i] = y * c + x * s;
+              for (int i4 = 0; i4 < 8; ++i4) {
+                const float4 c4 = __ldg(cs + i4), s4 = __ldg(sn + i4);
+                const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int i = 4 * i4 + e;
+                  const float x = __uint_as_float(ra[i]), y = __uint_as_float(rb[i]);
+                  a[i] = x * cv[e] - y * sv[e];
+                  b[i] = y * cv[e] + x * sv[e];
+                }
               }
             } else {
 #pragma unroll
@@ -233,12 +248,37 @@ __global__ void __launch_bounds__(THREADS, 1)
             store_bf16x32(dst + 64 + half * 32, b);
           }
         }
+      } else if (EPI == EPI_RESID) {
+        // unrolled so the two residual buffers stay in registers
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          if (live && c + 1 < BN / 32) {
+            const float4* src = reinterpret_cast<const float4*>((const float*)args.C + (size_t)row * args.ldc +
+                                                                n0 + (c + 1) * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) res[(c + 1) & 1][q] = src[q];
+          }
+          uint32_t r[32];
+          tmem_ld32(tbase + c * 32, r);
+          tmem_wait_ld(r);
+          if (!live) continue;
+          float4* d = reinterpret_cast<float4*>((float*)args.C + (size_t)row * args.ldc + n0 + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 x = res[c & 1][q];
+            x.x += __uint_as_float(r[4 * q]);
+            x.y += __uint_as_float(r[4 * q + 1]);
+            x.z += __uint_as_float(r[4 * q + 2]);
+            x.w += __uint_as_float(r[4 * q + 3]);
+            d[q] = x;
+          }
+        }
       } else {
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
           tmem_ld32(tbase + c * 32, r);
           tmem_wait_ld(r);
-          if (row >= args.M) continue;
+          if (!live) continue;
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
@@ -247,17 +287,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             float4* d = reinterpret_cast<float4*>((float*)args.C + (size_t)row * args.ldc + col);
 #pragma unroll
             for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          } else if (EPI == EPI_RESID) {
-            float4* d = reinterpret_cast<float4*>((float*)args.C + (size_t)row * args.ldc + col);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              float4 x = d[q];
-              x.x += v[4 * q];
-              x.y += v[4 * q + 1];
-              x.z += v[4 * q + 2];
-              x.w += v[4 * q + 3];
-              d[q] = x;
-            }
           } else {
             if (EPI == EPI_GELU) {
 #pragma unroll

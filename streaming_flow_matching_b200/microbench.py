@@ -4,6 +4,7 @@
   python -m streaming_flow_matching_b200.microbench append [--layers 28 --units 1]
   python -m streaming_flow_matching_b200.microbench euler [--n 268435456]
   python -m streaming_flow_matching_b200.microbench linear --m 924 --n 12288 --k 3072 [--epilogue gelu]
+  python -m streaming_flow_matching_b200.microbench step [--layers 1 --cache-units 4]
   python -m streaming_flow_matching_b200.microbench sweep      # attention + append sweep
 
 Inputs are seeded and larger than L2 where the case allows; each timing is
@@ -110,9 +111,29 @@ def bench_euler(n, warmup, reps):
             "peak_source": src}
 
 
+def bench_step(layers, cache_units, warmup, reps):
+    """One Euler step (denoise_step) at the 640x368 unit width with `layers` layers and a
+    `cache_units`-unit cache: a small-memory stand-in for ncu captures of the step's kernels."""
+    w = S.V02.replace(name=f"v0.2-width-{layers}L", n_layers=layers, cache_units=cache_units)
+    dev = torch.device("cuda", 0)
+    weights = S.make_weights(w, device=dev)
+    pool = cache_units * w.unit_kv_tokens + w.n_tokens
+    p = Performer.from_workload(w, weights, pool_tokens=pool, max_sessions=1)
+    s_id = p.open_session(cache_units)
+    k, v = S.make_kv_slices(w, cache_units, device=dev)
+    p.kvcache_append(s_id, k, v)
+    _, eps = S.make_latents(w, device=dev)
+    z = eps[0].clone()
+    ms = _time(lambda: p.denoise_step(s_id, z, 1.0, 0.75), warmup, reps)
+    p.check_device_error()
+    return {"case": "step", "layers": layers, "cache_tokens": cache_units * w.unit_kv_tokens,
+            "ms": ms}
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attention", "append", "euler", "linear", "sweep"])
+    ap.add_argument("case", choices=["attention", "append", "euler", "linear", "step", "sweep"])
+    ap.add_argument("--cache-units", type=int, default=4)
     ap.add_argument("--m", type=int, default=924)
     ap.add_argument("--k", type=int, default=3072)
     ap.add_argument("--epilogue", default="gelu")
@@ -135,6 +156,8 @@ def main():
         out.append(bench_euler(a.n, a.warmup, a.reps))
     elif a.case == "linear":
         out.append(bench_linear(a.m, a.n, a.k, a.epilogue, a.warmup, a.reps))
+    elif a.case == "step":
+        out.append(bench_step(a.layers, a.cache_units, a.warmup, a.reps))
     else:
         for m, n, k, e in [(924, 9216, 3072, "f32"), (924, 3072, 3072, "resid"),
                            (924, 12288, 3072, "gelu"), (924, 3072, 12288, "resid")]:

@@ -11,6 +11,8 @@ FP32_TOL = 1e-5     # relative L2 in the fp32 mode
 # small bf16 case the oracle finishes in well under a second: several query
 # tiles with a ragged tail (204 = 3 x 64 + 12), ragged key tiles (500 + 204 keys)
 SMALL_BF16 = S.Workload("small-bf16", 2, 512, 4, 128, 2048, 16, 200, 4, 100, 5, 4, "bf16")
+# d_model above 4096 (RMSNorm rows of 528 threads, 33 head-kernel column groups per thread)
+WIDE_BF16 = S.Workload("wide-bf16", 1, 4224, 2, 128, 256, 16, 24, 4, 32, 3, 2, "bf16")
 
 
 def ocfg(w):

@@ -12,8 +12,8 @@ import torch
 
 import sfm_synth as S
 from oracle import sfm_oracle as O
-from tests._gpu_util import (BF16_TOL, FP32_TOL, SMALL_BF16, ocfg, oracle_cache_layers, rel_l2,
-                             to_cuda, tol)
+from tests._gpu_util import (BF16_TOL, FP32_TOL, SMALL_BF16, WIDE_BF16, ocfg, oracle_cache_layers,
+                             rel_l2, to_cuda, tol)
 
 pytestmark = pytest.mark.gpu
 
@@ -49,7 +49,7 @@ def _oracle_velocity(w, weights_cpu, k, v, n_units, eps, tau):
 # whole-step and whole-solve parity
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("w", [S.TINY, SMALL_BF16], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [S.TINY, SMALL_BF16, WIDE_BF16], ids=lambda w: w.name)
 def test_velocity_and_solve_match_oracle(cuda_device, w):
     weights_cpu, weights, k, v, p, s = _setup(w)
     z0, eps = S.make_latents(w)

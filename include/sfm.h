@@ -184,6 +184,19 @@ SFM_API int sfm_fm_solve(sfm_handle* h, int session, float* z, const float* taus
 SFM_API int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions,
                          float* const* z, const float* taus, int n_taus, void* stream);
 
+/*
+ * Launch mode of sfm_denoise_step / sfm_fm_solve / sfm_fm_solve_batched.
+ * enabled = 1 (the default): each call is captured into one CUDA graph on a
+ * stream private to the handle and the graph is launched on the caller's
+ * stream (the handle keeps the executable graph and updates it in place on
+ * the next call).  enabled = 0: kernels are launched directly on the
+ * caller's stream.  Results are identical in both modes.  A call made while
+ * sfm_profile_begin is in effect launches directly (the profiler brackets
+ * every launch with events).  SFM_EINVAL for other values.  No counterpart
+ * in the method's description: a launch mechanism.
+ */
+SFM_API int sfm_set_graph_mode(sfm_handle* h, int enabled);
+
 /* ---- standalone kernels --------------------------------------------------- */
 
 /*

@@ -34,6 +34,10 @@ struct sfm_handle {
   std::vector<const void*> g_attn, w_qkv, w_o, g_mlp, w_1, w_2;
   void* k_pool = nullptr;
   void* v_pool = nullptr;
+  // solves run as one CUDA graph, captured on a private stream and updated in place
+  bool graphs = true;
+  cudaStream_t cap_stream = nullptr;
+  cudaGraphExec_t graph_exec = nullptr;
   long long pool_used = 0;
   std::vector<Session> sessions;
   // scratch, sized for max_sessions * n_tok rows
@@ -277,8 +281,8 @@ int check_taus(const float* taus, int n_taus) {
   return SFM_OK;
 }
 
-int solve(sfm_handle* h, int n, const int* sessions, float* const* z, const float* taus,
-          int n_taus, float* const* v_out, cudaStream_t s) {
+int solve_direct(sfm_handle* h, int n, const int* sessions, float* const* z, const float* taus,
+                 int n_taus, float* const* v_out, cudaStream_t s) {
   BatchDesc b;
   fill_batch(h, n, sessions, &b);
   int rc;
@@ -292,6 +296,45 @@ int solve(sfm_handle* h, int n, const int* sessions, float* const* z, const floa
     if (rc) return rc;
   }
   return SFM_OK;
+}
+
+// A solve is several hundred small launches (8 per layer per Euler step).  They
+// are captured into a graph on the handle's private stream and the graph is
+// launched on the caller's stream; the executable graph is kept and updated in
+// place from each new capture (same topology, new kernel arguments: positions,
+// cache lengths, latent pointers), so repeated units pay neither instantiation
+// nor per-launch overheads.  The profiler brackets every launch with events,
+// so a profiled call launches directly.
+int solve(sfm_handle* h, int n, const int* sessions, float* const* z, const float* taus,
+          int n_taus, float* const* v_out, cudaStream_t s) {
+  if (!h->graphs || !h->cap_stream || profiling_active())
+    return solve_direct(h, n, sessions, z, taus, n_taus, v_out, s);
+  if (cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
+    return record_cuda(cudaGetLastError());
+  const int rc = solve_direct(h, n, sessions, z, taus, n_taus, v_out, h->cap_stream);
+  cudaGraph_t g = nullptr;
+  const cudaError_t ec = cudaStreamEndCapture(h->cap_stream, &g);
+  if (rc || ec != cudaSuccess || !g) {
+    if (g) cudaGraphDestroy(g);
+    cudaGetLastError();
+    return rc ? rc : record_cuda(ec != cudaSuccess ? ec : cudaErrorStreamCaptureInvalidated);
+  }
+  if (h->graph_exec) {
+    cudaGraphExecUpdateResultInfo info;
+    if (cudaGraphExecUpdate(h->graph_exec, g, &info) != cudaSuccess) {
+      cudaGetLastError();
+      cudaGraphExecDestroy(h->graph_exec);
+      h->graph_exec = nullptr;
+    }
+  }
+  cudaError_t e = cudaSuccess;
+  if (!h->graph_exec) e = cudaGraphInstantiate(&h->graph_exec, g, 0);
+  cudaGraphDestroy(g);
+  if (e != cudaSuccess) {
+    h->graph_exec = nullptr;
+    return record_cuda(e);
+  }
+  return record_cuda(cudaGraphLaunch(h->graph_exec, s));
 }
 
 }  // namespace
@@ -379,6 +422,11 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     int dev = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, dev);
+    // a handle without its capture stream still works, with direct launches
+    if (cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaGetLastError();
+      h->cap_stream = nullptr;
+    }
   }
   if (!rc && h->has_weights && cfg->dtype == SFM_DTYPE_BF16) {
     const int L_ = cfg->n_layers, d_ = cfg->d_model, hd_ = h->hd, F_ = cfg->d_mlp;
@@ -420,6 +468,8 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
 void sfm_destroy(sfm_handle* h) {
   if (!h) return;
   cudaDeviceSynchronize();
+  if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   for (void* p : h->owned) cudaFree(p);
   delete h;
 }
@@ -515,6 +565,17 @@ int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long long row0
     return SFM_EINVAL;
   return launch_kv_read(h->k_pool, h->v_pool, k_dst, v_dst, layer, h->cfg.pool_tokens,
                         h->hd * h->es, s.base_row + row0, n_rows, (cudaStream_t)stream);
+}
+
+int sfm_set_graph_mode(sfm_handle* h, int enabled) {
+  if (!h || (enabled != 0 && enabled != 1)) return SFM_EINVAL;
+  h->graphs = enabled != 0;
+  if (!h->graphs && h->graph_exec) {
+    // launches already enqueued keep their copy of the graph
+    cudaGraphExecDestroy(h->graph_exec);
+    h->graph_exec = nullptr;
+  }
+  return SFM_OK;
 }
 
 int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_from, float tau_to,

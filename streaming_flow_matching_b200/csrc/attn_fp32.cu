@@ -49,6 +49,8 @@ __global__ void attn_f32_kernel(AttnDesc a, const float* __restrict__ q,
 }
 
 // Merge split-KV partials: one warp per (row, head); D = 128 (float4 per lane).
+// Every split's log-sum-exp and partial row are loaded up front, so the loads
+// of a row are in flight together.
 __global__ void attn_merge_kernel(const float* __restrict__ o_part,
                                   const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ o,
                                   long long total_rows, int H, int n_splits) {
@@ -57,23 +59,34 @@ __global__ void attn_merge_kernel(const float* __restrict__ o_part,
   if (gw >= total_rows * H) return;
   const long long row = gw / H;
   const int h = (int)(gw - row * H);
+  const long long ld = (long long)H * 128;
+  float lse[kMaxSplits];
+  float4 p[kMaxSplits];
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    if (s < n_splits) {
+      lse[s] = __ldcs(lse_part + ((long long)s * total_rows + row) * H + h);
+      p[s] = __ldcs(reinterpret_cast<const float4*>(o_part + ((long long)s * total_rows + row) * ld +
+                                                    h * 128) + lane);
+    } else {
+      lse[s] = -INFINITY;
+      p[s] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
   float mmax = -INFINITY;
-  for (int s = 0; s < n_splits; ++s)
-    mmax = fmaxf(mmax, lse_part[((long long)s * total_rows + row) * H + h]);
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) mmax = fmaxf(mmax, lse[s]);
   float wsum = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const long long ld = (long long)H * 128;
-  for (int s = 0; s < n_splits; ++s) {
-    const float lse = lse_part[((long long)s * total_rows + row) * H + h];
-    if (lse == -INFINITY) continue;
-    const float w = exp2f(lse - mmax);
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    // a split without keys has lse = -inf and weight 0 (its partial row is zeros)
+    const float w = lse[s] == -INFINITY ? 0.f : exp2f(lse[s] - mmax);
     wsum += w;
-    const float4 p = reinterpret_cast<const float4*>(o_part + ((long long)s * total_rows + row) * ld +
-                                                     h * 128)[lane];
-    acc.x = fmaf(w, p.x, acc.x);
-    acc.y = fmaf(w, p.y, acc.y);
-    acc.z = fmaf(w, p.z, acc.z);
-    acc.w = fmaf(w, p.w, acc.w);
+    acc.x = fmaf(w, p[s].x, acc.x);
+    acc.y = fmaf(w, p[s].y, acc.y);
+    acc.z = fmaf(w, p[s].z, acc.z);
+    acc.w = fmaf(w, p[s].w, acc.w);
   }
   const float inv = 1.f / wsum;
   __nv_bfloat16* od = o + row * ld + h * 128 + lane * 4;

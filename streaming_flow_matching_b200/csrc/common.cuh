@@ -39,6 +39,10 @@ void count_launch();             // one more kernel launched by this library
 
 // Records a CUDA event pair around the launches in its scope when the
 // profiler is on (sfm_profile_begin); no-op otherwise.
+// True while sfm_profile_begin is in effect on this thread (launches are then
+// issued directly, each bracketed by events, instead of through a CUDA graph).
+bool profiling_active();
+
 class ProfScope {
  public:
   ProfScope(int kind, cudaStream_t s);

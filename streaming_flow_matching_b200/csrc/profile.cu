@@ -19,6 +19,10 @@ std::atomic<unsigned long long> g_launches{0};
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+bool profiling_active() { return g_prof.on; }
+
+
+
 ProfScope::ProfScope(int kind, cudaStream_t s) : s_(s) {
   if (!g_prof.on || g_prof.used * 2 + 1 >= (int)g_prof.ev.size()) return;
   idx_ = g_prof.used++;

@@ -136,6 +136,10 @@ class Performer:
         L.check(L.lib.sfm_fm_solve_batched(self._h, n, s, zp, t, len(taus), _stream()),
                 "sfm_fm_solve_batched")
 
+    def set_graph_mode(self, enabled):
+        """Solves as one captured CUDA graph (True, the default) or direct launches."""
+        L.check(L.lib.sfm_set_graph_mode(self._h, 1 if enabled else 0), "sfm_set_graph_mode")
+
     def check_device_error(self):
         """Synchronises and returns the handle's device error word (0 = no kernel problem)."""
         code = C.c_int()

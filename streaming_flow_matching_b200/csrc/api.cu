@@ -58,6 +58,7 @@ struct sfm_handle {
   CUtensorMap map_q{}, map_kpool{}, map_vpool{};  // attention operands
   std::vector<CUtensorMap> map_wqkv, map_wo, map_w1, map_w2;
   int bn_qkv = 0, bn_o = 0, bn_up = 0, bn_down = 0;   // N-tile widths the weight maps use
+  bool pair_qkv = false, pair_o = false, pair_up = false, pair_down = false;   // CTA pairs
   std::vector<void*> owned;
 
   void* layer_k(int l) const { return (char*)k_pool + (size_t)l * cfg.pool_tokens * hd * es; }
@@ -163,7 +164,8 @@ int make_rows_map(CUtensorMap* m, const void* p, long long rows, int heads, int 
   return make_tmap_bf16(m, p, 3, dims, strides, box);
 }
 
-GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err, int block_n = 0) {
+GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err, int block_n,
+                   bool pair) {
   GemmArgs g{};
   g.M = M;
   g.N = N;
@@ -174,6 +176,7 @@ GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err, int
   g.err = err;
   g.hd = 0;
   g.block_n = block_n;
+  g.pair = pair ? 1 : 0;
   return g;
 }
 
@@ -206,7 +209,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
     if (tc) {
       // QKV projection with RoPE and the cache-tail scatter fused in the epilogue
       ProfScope ps(SFM_PROF_GEMM_QKV, s);
-      GemmArgs g = gemm_args(M, 3 * hd, d, EPI_QKV, nullptr, 0, h->d_err);
+      GemmArgs g = gemm_args(M, 3 * hd, d, EPI_QKV, nullptr, 0, h->d_err, h->bn_qkv, h->pair_qkv);
       g.cos_t = h->cos_t;
       g.sin_t = h->sin_t;
       g.q_out = (__nv_bfloat16*)h->q;
@@ -214,7 +217,6 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       g.v_layer = (__nv_bfloat16*)h->layer_v(l);
       g.hd = hd;
       g.b = b;
-      g.block_n = h->bn_qkv;
       SFM_TRY(launch_gemm_tc(h->map_xn, h->map_wqkv[l], g, h->sms, s));
     } else {
       {
@@ -237,7 +239,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_O, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_ao, h->map_wo[l],
-                               gemm_args(M, d, hd, EPI_RESID, h->x, d, h->d_err, h->bn_o), h->sms, s));
+                               gemm_args(M, d, hd, EPI_RESID, h->x, d, h->d_err, h->bn_o, h->pair_o), h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->ao, h->w_o[l], h->x, M, d, hd, EPI_RESID, dt, s));
       }
@@ -250,7 +252,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_UP, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_xn, h->map_w1[l],
-                               gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->d_err, h->bn_up), h->sms, s));
+                               gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->d_err, h->bn_up, h->pair_up), h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->xn, h->w_1[l], h->hmlp, M, F, d, EPI_GELU, dt, s));
       }
@@ -259,7 +261,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_DOWN, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_hmlp, h->map_w2[l],
-                               gemm_args(M, d, F, EPI_RESID, h->x, d, h->d_err, h->bn_down), h->sms, s));
+                               gemm_args(M, d, F, EPI_RESID, h->x, d, h->d_err, h->bn_down, h->pair_down), h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->hmlp, h->w_2[l], h->x, M, d, F, EPI_RESID, dt, s));
       }
@@ -444,17 +446,24 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     h->map_wo.resize(L_);
     h->map_w1.resize(L_);
     h->map_w2.resize(L_);
-    // tile widths chosen for a full batch (max_sessions units)
-    h->bn_qkv = gemm_tc_block_n((int)M, 3 * hd_, hd_, EPI_QKV, h->sms);
-    h->bn_o = gemm_tc_block_n((int)M, d_, 0, EPI_RESID, h->sms);
-    h->bn_up = gemm_tc_block_n((int)M, F_, 0, EPI_GELU, h->sms);
-    h->bn_down = gemm_tc_block_n((int)M, d_, 0, EPI_RESID, h->sms);
+    // mode and tile widths chosen for a full batch (max_sessions units); the weight
+    // maps' boxes depend on both
+    const int mm = (int)M;
+    h->pair_qkv = gemm_tc_pair(mm, 3 * hd_, hd_, EPI_QKV, h->sms);
+    h->pair_o = gemm_tc_pair(mm, d_, 0, EPI_RESID, h->sms);
+    h->pair_up = gemm_tc_pair(mm, F_, 0, EPI_GELU, h->sms);
+    h->pair_down = gemm_tc_pair(mm, d_, 0, EPI_RESID, h->sms);
+    h->bn_qkv = gemm_tc_block_n(mm, 3 * hd_, hd_, EPI_QKV, h->sms, h->pair_qkv);
+    h->bn_o = gemm_tc_block_n(mm, d_, 0, EPI_RESID, h->sms, h->pair_o);
+    h->bn_up = gemm_tc_block_n(mm, F_, 0, EPI_GELU, h->sms, h->pair_up);
+    h->bn_down = gemm_tc_block_n(mm, d_, 0, EPI_RESID, h->sms, h->pair_down);
     if (!h->bn_qkv || !h->bn_o || !h->bn_up || !h->bn_down) rc = SFM_EUNSUPPORTED;
+    // the B box holds the weight rows one CTA stages: half the tile on pairs
     for (int l = 0; l < L_ && !rc; ++l) {
-      rc = make_b_map(&h->map_wqkv[l], h->w_qkv[l], 3 * hd_, d_, h->bn_qkv);
-      if (!rc) rc = make_b_map(&h->map_wo[l], h->w_o[l], d_, hd_, h->bn_o);
-      if (!rc) rc = make_b_map(&h->map_w1[l], h->w_1[l], F_, d_, h->bn_up);
-      if (!rc) rc = make_b_map(&h->map_w2[l], h->w_2[l], d_, F_, h->bn_down);
+      rc = make_b_map(&h->map_wqkv[l], h->w_qkv[l], 3 * hd_, d_, h->bn_qkv / (h->pair_qkv ? 2 : 1));
+      if (!rc) rc = make_b_map(&h->map_wo[l], h->w_o[l], d_, hd_, h->bn_o / (h->pair_o ? 2 : 1));
+      if (!rc) rc = make_b_map(&h->map_w1[l], h->w_1[l], F_, d_, h->bn_up / (h->pair_up ? 2 : 1));
+      if (!rc) rc = make_b_map(&h->map_w2[l], h->w_2[l], d_, F_, h->bn_down / (h->pair_down ? 2 : 1));
     }
   }
   if (rc) {
@@ -695,13 +704,15 @@ int sfm_linear(const void* x, const void* w, void* y, int M, int N, int K, int e
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int bn = gemm_tc_block_n(M, N, 0, epi, sms);
+  const bool pair = gemm_tc_pair(M, N, 0, epi, sms);
+  const int bn = gemm_tc_block_n(M, N, 0, epi, sms, pair);
   if (!bn) return SFM_EUNSUPPORTED;
   CUtensorMap ma, mb;
   int rc = make_a_map(&ma, x, M, K);
-  if (!rc) rc = make_b_map(&mb, w, N, K, bn);
+  if (!rc) rc = make_b_map(&mb, w, N, K, pair ? bn / 2 : bn);
   if (rc) return rc;
-  return launch_gemm_tc(ma, mb, gemm_args(M, N, K, epi, y, N, nullptr, bn), sms, (cudaStream_t)stream);
+  return launch_gemm_tc(ma, mb, gemm_args(M, N, K, epi, y, N, nullptr, bn, pair), sms,
+                        (cudaStream_t)stream);
 }
 
 const char* sfm_strerror(int status) {

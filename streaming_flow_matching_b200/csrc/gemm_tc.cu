@@ -10,6 +10,14 @@
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (thread = row), fused
 //               epilogue, global stores; the other accumulator is being filled
 //               meanwhile
+// Pair mode (two CTAs of a cluster on neighbouring SMs, tcgen05 cta_group::2):
+// a 256-row tile, rows [0,128) in the even CTA and [128,256) in the odd one; each
+// CTA stages its own A rows and half of the B tile (BN/2 weight rows), so every
+// weight byte reaches shared memory once per pair instead of once per CTA.  Both
+// CTAs' loads of a stage complete on the even CTA's barrier (which expects the
+// bytes of both); the even CTA's lane issues the M = 256 MMAs and its commits
+// arrive on both CTAs' barriers; each CTA's epilogue drains its own 128
+// accumulator rows.
 // Epilogues: EPI_F32 / EPI_STORE / EPI_GELU / EPI_RESID (x += acc, fp32) and
 // EPI_QKV: rotary embedding of q and k in fp32 (rotate-half pairs (i, i+64) of
 // each 128-wide head), q to the Q buffer, k and v to the sessions' cache rows
@@ -26,10 +34,12 @@ namespace gtc {
 constexpr int BM = 128, BK = 64;
 constexpr int THREADS = 192;
 
-template <int BN> struct Cfg {
-  static constexpr int STAGES = BN == 256 ? 4 : (BN == 192 ? 5 : 6);
+template <int BN, bool PAIR> struct Cfg {
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;   // weight rows staged by this CTA
+  static constexpr int STAGES = PAIR ? (BN == 256 ? 6 : (BN == 192 ? 7 : 8))
+                                     : (BN == 256 ? 4 : (BN == 192 ? 5 : 6));
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int ACC_COLS = BN == 128 ? 128 : 256;     // TMEM columns between the two accumulators
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
@@ -54,11 +64,12 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a,
                    const __grid_constant__ CUtensorMap map_b, const __grid_constant__ GemmArgs args) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, PAIR>;
+  static_assert(C::STAGES <= 8, "producer bookkeeping holds 8 stages");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -72,7 +83,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m_tiles = (args.M + BM - 1) / BM;
+  // tiles of TM rows: 128 (one CTA) or 256 (a pair); unit = this CTA or pair
+  constexpr int TM = PAIR ? 2 * BM : BM;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int m_tiles = (args.M + TM - 1) / TM;
   const int n_tiles = args.N / BN;
   const int tiles = m_tiles * n_tiles;
   const int kblocks = args.K / BK;
@@ -84,44 +101,63 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 128);
+      mbar_init(&acc_empty[a], PAIR ? 8 : 4);   // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     *abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch(&map_a);
     tma_prefetch(&map_b);
   }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) {
+    __syncwarp();
+    cluster_sync();        // both CTAs' barriers exist before any remote arrive
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer ----------------
+      // ---------------- TMA producer (its own A rows and B rows) ----------------
       int s = 0;
       uint32_t ph = 0;
       int last_parity[8];
       for (int i = 0; i < C::STAGES; ++i) last_parity[i] = -1;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        const int m0 = (t % m_tiles) * BM, n0 = (t / m_tiles) * BN;
+      for (int t = unit; t < tiles && ok; t += n_units) {
+        const int m0 = (t % m_tiles) * TM + (int)rank * BM;
+        const int n0 = (t / m_tiles) * BN + (int)rank * C::B_ROWS;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort, args.err, 0x101)) {
             ok = false;
             break;
           }
           const uint32_t sa = base + s * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-          tma_load_2d(sa, &map_a, &full[s], kb * BK, m0);
-          tma_load_2d(sa + C::A_BYTES, &map_b, &full[s], kb * BK, n0);
+          if (PAIR) {
+            // both halves complete on the even CTA's barrier, which expects both
+            const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE_BYTES);
+            tma_load_2d_pair(sa, &map_a, bar, kb * BK, m0);
+            tma_load_2d_pair(sa + C::A_BYTES, &map_b, bar, kb * BK, n0);
+          } else {
+            mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+            tma_load_2d(sa, &map_a, &full[s], kb * BK, m0);
+            tma_load_2d(sa + C::A_BYTES, &map_b, &full[s], kb * BK, n0);
+          }
           last_parity[s] = (int)ph;
           if (++s == C::STAGES) {
             s = 0;
@@ -129,21 +165,30 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (!ok)  // unwinding: let the loads already issued land before the CTA exits
-        for (int i = 0; i < C::STAGES; ++i)
-          if (last_parity[i] >= 0) mbar_drain(&full[i], (uint32_t)last_parity[i]);
+      if (!ok) {  // unwinding: let the loads already issued land before the CTA exits
+        if (PAIR && !leader) {
+          // this CTA's loads complete on the even CTA's barrier: give them a bound
+          const unsigned long long t0 = globaltimer();
+          while (globaltimer() - t0 < 100000ull) {
+          }
+        } else {
+          for (int i = 0; i < C::STAGES; ++i)
+            if (last_parity[i] >= 0) mbar_drain(&full[i], (uint32_t)last_parity[i]);
+        }
+      }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = idesc_bf16(BM, BN, false, false);
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (the CTA, or the pair's even CTA) ----------------
+      constexpr uint32_t idesc = idesc_bf16(TM, BN, false, false);
       int s = 0;
       uint32_t ph = 0;
       int acc = 0;
       uint32_t acc_ph = 0;
       bool ok = true, issued = false;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102)) {
+      for (int t = unit; t < tiles && ok; t += n_units) {
+        if (!(PAIR ? mbar_wait_cluster(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102)
+                   : mbar_wait(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102))) {
           ok = false;
           break;
         }
@@ -159,23 +204,37 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint64_t da = sw128_desc(sa, 16, 1024);
           const uint64_t db = sw128_desc(sa + C::A_BYTES, 16, 1024);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)  // +32 bytes per K=16 step inside the swizzle atom
-            umma_bf16(d, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
-                      (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < BK / 16; ++k) {  // +32 bytes per K=16 step inside the swizzle atom
+            if (PAIR)
+              umma_bf16_pair(d, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
+                             (kb | k) != 0 ? 1u : 0u);
+            else
+              umma_bf16(d, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
+                        (kb | k) != 0 ? 1u : 0u);
+          }
           issued = true;
-          umma_commit(&empty[s]);
+          if (PAIR)
+            umma_commit_pair(&empty[s], 3);
+          else
+            umma_commit(&empty[s]);
           if (++s == C::STAGES) {
             s = 0;
             ph ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(&acc_full[acc]);
+        if (PAIR)
+          umma_commit_pair(&acc_full[acc], 3);
+        else
+          umma_commit(&acc_full[acc]);
         acc ^= 1;
         if (acc == 0) acc_ph ^= 1u;
       }
       if (!ok && issued) {  // unwinding: wait for the MMAs already issued
-        umma_commit(drain);
+        if (PAIR)
+          umma_commit_pair(drain, 1);
+        else
+          umma_commit(drain);
         mbar_drain(drain, 0);
       }
     }
@@ -184,8 +243,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;              // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_ph = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x) {
-      const int m0 = (t % m_tiles) * BM, n0 = (t / m_tiles) * BN;
+    for (int t = unit; t < tiles; t += n_units) {
+      const int m0 = (t % m_tiles) * TM + (int)rank * BM, n0 = (t / m_tiles) * BN;
       const int row = m0 + quarter * 32 + lane;
       const bool live = row < args.M;
       // residual add: this row's fp32 slice of chunk 0 is loaded (from L2) while the
@@ -196,7 +255,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int q = 0; q < 8; ++q) res[0][q] = src[q];
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[acc], acc_ph, abort, args.err, 0x104))) break;
+      if (!__all_sync(0xffffffffu, PAIR ? mbar_wait_cluster(&acc_full[acc], acc_ph, abort, args.err, 0x104)
+                                        : mbar_wait(&acc_full[acc], acc_ph, abort, args.err, 0x104)))
+        break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
       if (EPI == EPI_QKV) {
@@ -297,39 +358,83 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[acc]);
+      __syncwarp();
+      if (lane == 0) {
+        if (PAIR)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
+        else
+          mbar_arrive(&acc_empty[acc]);
+      }
       acc ^= 1;
       if (acc == 0) acc_ph ^= 1u;
     }
   }
 
+  // neither CTA of a pair frees its TMEM or exits while the pair's MMAs, loads or
+  // remote arrivals may still touch it
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) {
+    __syncwarp();
+    cluster_sync();
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if (PAIR)
+      tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool PAIR>
 int launch_bn(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,
               cudaStream_t s) {
-  using C = Cfg<BN>;
-  const int tiles = ((args.M + BM - 1) / BM) * (args.N / BN);
-  const int grid = tiles < sms ? tiles : sms;
-  cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       C::SMEM);
-  gemm_tc_kernel<BN, EPI><<<grid, THREADS, C::SMEM, s>>>(a, b, args);
-  return record_cuda(cudaGetLastError());
+  using C = Cfg<BN, PAIR>;
+  constexpr int TM = PAIR ? 2 * BM : BM;
+  const int tiles = ((args.M + TM - 1) / TM) * (args.N / BN);
+  const int units = PAIR ? sms / 2 : sms;
+  const int grid = (tiles < units ? tiles : units) * (PAIR ? 2 : 1);
+  auto kern = gemm_tc_kernel<BN, EPI, PAIR>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = PAIR ? 1 : 0;
+  return record_cuda(cudaLaunchKernelEx(&cfg, kern, a, b, args));
 }
 
 }  // namespace gtc
 
-int gemm_tc_block_n(int M, int N, int hd, int epi, int sms) {
+bool gemm_tc_pair(int M, int N, int hd, int epi, int sms) {
+  // Pairs halve each SM's weight traffic but add a cross-SM hop to every stage;
+  // they pay off when every pair has several tiles to pipeline (measured on the
+  // 924-row projections: +4-5 % for N = 9216 and 12288 at 2-2.6 tiles per pair,
+  // -6-8 % for N = 3072 at under one).
+  if (M <= gtc::BM || sms < 2) return false;
+  const int bn = gemm_tc_block_n(M, N, hd, epi, sms, true);
+  if (!bn) return false;
+  const long long tiles = (long long)((M + 2 * gtc::BM - 1) / (2 * gtc::BM)) * (N / bn);
+  return 2 * tiles >= 3LL * (sms / 2);
+}
+
+int gemm_tc_block_n(int M, int N, int hd, int epi, int sms, bool pair) {
   // N-tile width minimising (waves of the persistent grid) x (work per tile);
   // ties go to the wider tile.  The QKV epilogue works on whole 128-wide heads.
+  // Pairs take 256-row tiles and run on sms / 2 units.
   const int cands[3] = {256, 192, 128};
-  const long long m_tiles = (M + gtc::BM - 1) / gtc::BM;
+  if (pair) sms /= 2;
+  const int tm = pair ? 2 * gtc::BM : gtc::BM;
+  const long long m_tiles = (M + tm - 1) / tm;
   int best = 0;
   long long best_cost = 0;
   for (int bn : cands) {
@@ -348,11 +453,15 @@ int gemm_tc_block_n(int M, int N, int hd, int epi, int sms) {
 int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,
                    cudaStream_t s) {
   if (args.M <= 0) return SFM_OK;
-  const int bn = args.block_n ? args.block_n : gemm_tc_block_n(args.M, args.N, args.hd, args.epi, sms);
+  const bool pair = args.pair != 0;
+  if (pair && sms < 2) return SFM_EUNSUPPORTED;
+  const int bn = args.block_n;
   if (!bn || args.N % bn || args.K % gtc::BK || args.K <= 0) return SFM_EUNSUPPORTED;
   if (args.epi == EPI_QKV && (args.hd % bn || args.N != 3 * args.hd)) return SFM_EUNSUPPORTED;
-#define SFM_GTC(BN_, E)                                          \
-  if (bn == BN_ && args.epi == E) return gtc::launch_bn<BN_, E>(a, b, args, sms, s);
+#define SFM_GTC(BN_, E)                                                              \
+  if (bn == BN_ && args.epi == E)                                                    \
+    return pair ? gtc::launch_bn<BN_, E, true>(a, b, args, sms, s)                  \
+                : gtc::launch_bn<BN_, E, false>(a, b, args, sms, s);
   SFM_GTC(256, EPI_F32)
   SFM_GTC(256, EPI_GELU)
   SFM_GTC(256, EPI_RESID)

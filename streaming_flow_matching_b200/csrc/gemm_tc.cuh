@@ -20,12 +20,18 @@ struct GemmArgs {
   __nv_bfloat16* v_layer;
   int hd;
   BatchDesc b;
-  int block_n;           // N-tile width the B tensor map was built for (0: choose)
+  int block_n;           // N-tile width the B tensor map was built for
+  int pair;              // 1: CTA pairs (the B map's box has block_n / 2 rows)
 };
 
-// N-tile width (256, 192 or 128) for an M x N problem on `sms` SMs; 0 if none fits.
-int gemm_tc_block_n(int M, int N, int hd, int epi, int sms);
-// A: tensor map over [M_alloc][K] bf16, box {64, 128}; B: over [N][K], box {64, block_n}.
+// Whether an M x N projection runs on CTA pairs (256-row tiles, half of each B
+// tile per CTA): M above 128 and at least 1.5 tiles per pair.
+bool gemm_tc_pair(int M, int N, int hd, int epi, int sms);
+// N-tile width (256, 192 or 128) for an M x N problem on `sms` SMs, in the given
+// mode; 0 if none fits.
+int gemm_tc_block_n(int M, int N, int hd, int epi, int sms, bool pair);
+// A: tensor map over [M_alloc][K] bf16, box {64, 128}; B: over [N][K], box
+// {64, pair ? block_n / 2 : block_n}.
 int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,
                    cudaStream_t s);
 

@@ -1,7 +1,7 @@
 """Dense projections through the C ABI (sfm_linear) against the oracle's
 matmul in fp64: tcgen05 tiles with ragged M tails, every N-tile width (128,
-192, 256: the width follows from M and N), every epilogue; fp32 mode on the
-CUDA cores."""
+192, 256: the width follows from M and N), single CTAs and CTA pairs, every
+epilogue; fp32 mode on the CUDA cores."""
 import numpy as np
 import pytest
 import torch
@@ -11,8 +11,10 @@ from tests._gpu_util import rel_l2
 
 pytestmark = pytest.mark.gpu
 
+# 924 x 9216 / 12288 run on CTA pairs (256-row tiles); 800 x 12288 leaves the odd CTA
+# of the last pair without rows
 SHAPES = [(1, 128, 64), (130, 256, 128), (300, 384, 192), (924, 3072, 3072), (924, 9216, 3072),
-          (924, 3072, 12288), (1848, 1024, 512)]
+          (924, 3072, 12288), (1848, 1024, 512), (800, 12288, 256)]
 
 
 def _inputs(M, N, K, dtype, seed):

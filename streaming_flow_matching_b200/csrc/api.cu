@@ -48,6 +48,7 @@ struct sfm_handle {
   void* ao = nullptr;        // [M][H D] attention output
   void* hmlp = nullptr;      // [M][F] GELU(MLP-up)
   float* cos_t = nullptr;    // [M][D/2]
+  float* ss = nullptr;       // [M][d / 128]: fused-RMSNorm partial sums of squares
   float* sin_t = nullptr;
   float* o_part = nullptr;   // [kMaxSplits][M][H][D]
   float* lse_part = nullptr; // [kMaxSplits][M][H]
@@ -192,24 +193,51 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
   do {                               \
     if ((rc = (call)) != SFM_OK) return rc; \
   } while (0)
+  const bool tc = dt == SFM_DTYPE_BF16;
+  // bf16 path: every RMSNorm before a projection is split between the kernel that
+  // last updates x (it writes bf16(x g) and per-tile sums of squares) and the
+  // projection's epilogue (it scales each row by 1 / rms)
+  const int ss_ld = (d + 127) / 128;
+  int ss_n = ss_ld;                 // partial sums per row left by the last producer
   {
     ProfScope ps(SFM_PROF_ROWOPS, s);
-    SFM_TRY(launch_embed(b, z, h->w_in, h->e_mod, tau_from, h->x, d, c.c_lat, dt, s));
+    if (tc)
+      SFM_TRY(launch_embed(b, z, h->w_in, h->e_mod, tau_from, h->x, d, c.c_lat, dt, s,
+                           h->g_attn[0], h->xn, h->ss, ss_ld));
+    else
+      SFM_TRY(launch_embed(b, z, h->w_in, h->e_mod, tau_from, h->x, d, c.c_lat, dt, s));
   }
+  auto normed = [&](GemmArgs g) {   // a consumer of the fused norm
+    g.ss_in = h->ss;
+    g.ss_n = ss_n;
+    g.ss_ld = ss_ld;
+    g.norm_d = d;
+    g.norm_eps = eps;
+    return g;
+  };
+  auto norm_next = [&](GemmArgs g, const void* gain, int bn) {   // a producer
+    if (!gain) return g;
+    g.g_next = (const __nv_bfloat16*)gain;
+    g.xg = (__nv_bfloat16*)h->xn;
+    g.ss_out = h->ss;
+    g.ss_ld = ss_ld;
+    ss_n = d / bn;
+    return g;
+  };
   const AttnDesc ad = attn_desc(b);
   long long max_keys = 0;
   for (int i = 0; i < b.n; ++i) max_keys = ad.nkeys[i] > max_keys ? ad.nkeys[i] : max_keys;
-  const bool tc = dt == SFM_DTYPE_BF16;
   const int splits = tc ? attention_tc_splits(b.n_tok, b.n, max_keys, c.n_heads, h->sms) : 1;
   for (int l = 0; l < c.n_layers; ++l) {
-    {
+    if (!tc) {
       ProfScope ps(SFM_PROF_ROWOPS, s);
       SFM_TRY(launch_rmsnorm(h->x, h->g_attn[l], h->xn, M, d, eps, dt, s));
     }
     if (tc) {
-      // QKV projection with RoPE and the cache-tail scatter fused in the epilogue
+      // QKV projection with the norm's 1 / rms, RoPE and the cache-tail scatter fused in
+      // the epilogue
       ProfScope ps(SFM_PROF_GEMM_QKV, s);
-      GemmArgs g = gemm_args(M, 3 * hd, d, EPI_QKV, nullptr, 0, h->d_err, h->bn_qkv, h->pair_qkv);
+      GemmArgs g = normed(gemm_args(M, 3 * hd, d, EPI_QKV, nullptr, 0, h->d_err, h->bn_qkv, h->pair_qkv));
       g.cos_t = h->cos_t;
       g.sin_t = h->sin_t;
       g.q_out = (__nv_bfloat16*)h->q;
@@ -239,12 +267,14 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_O, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_ao, h->map_wo[l],
-                               gemm_args(M, d, hd, EPI_RESID, h->x, d, h->d_err, h->bn_o, h->pair_o), h->sms, s));
+                               norm_next(gemm_args(M, d, hd, EPI_RESID, h->x, d, h->d_err, h->bn_o, h->pair_o),
+                                         h->g_mlp[l], h->bn_o),
+                               h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->ao, h->w_o[l], h->x, M, d, hd, EPI_RESID, dt, s));
       }
     }
-    {
+    if (!tc) {
       ProfScope ps(SFM_PROF_ROWOPS, s);
       SFM_TRY(launch_rmsnorm(h->x, h->g_mlp[l], h->xn, M, d, eps, dt, s));
     }
@@ -252,7 +282,8 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_UP, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_xn, h->map_w1[l],
-                               gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->d_err, h->bn_up, h->pair_up), h->sms, s));
+                               normed(gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->d_err, h->bn_up, h->pair_up)),
+                               h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->xn, h->w_1[l], h->hmlp, M, F, d, EPI_GELU, dt, s));
       }
@@ -261,7 +292,9 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_DOWN, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_hmlp, h->map_w2[l],
-                               gemm_args(M, d, F, EPI_RESID, h->x, d, h->d_err, h->bn_down, h->pair_down), h->sms, s));
+                               norm_next(gemm_args(M, d, F, EPI_RESID, h->x, d, h->d_err, h->bn_down, h->pair_down),
+                                         l + 1 < c.n_layers ? h->g_attn[l + 1] : nullptr, h->bn_down),
+                               h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->hmlp, h->w_2[l], h->x, M, d, F, EPI_RESID, dt, s));
       }
@@ -399,6 +432,7 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     if (!rc) rc = dalloc(h, &h->ao, M * hd * es);
     if (!rc) rc = dalloc(h, &h->hmlp, M * F * es);
     if (!rc) rc = dalloc(h, &h->cos_t, M * (cfg->head_dim / 2) * 4);
+    if (!rc) rc = dalloc(h, &h->ss, M * ((cfg->d_model + 127) / 128) * 4);
     if (!rc) rc = dalloc(h, &h->sin_t, M * (cfg->head_dim / 2) * 4);
     if (!rc && cfg->dtype == SFM_DTYPE_BF16) {
       rc = dalloc(h, &h->o_part, (size_t)kMaxSplits * M * hd * 4);

@@ -63,8 +63,11 @@ int launch_kv_read(const void* k_pool, const void* v_pool, void* k_dst, void* v_
                    long long pool_tokens, int row_bytes, long long row0, long long n_rows,
                    cudaStream_t s);
 
+// With g (bf16 only): also xg = bf16(x g) and per-row partial sums of squares
+// over 128-column blocks into ss ([rows][ss_ld]) -- the first RMSNorm, fused.
 int launch_embed(const BatchDesc& b, float* const* z, const void* w_in, const void* e_mod,
-                 float tau, float* x, int d, int c_lat, int dtype, cudaStream_t s);
+                 float tau, float* x, int d, int c_lat, int dtype, cudaStream_t s,
+                 const void* g = nullptr, void* xg = nullptr, float* ss = nullptr, int ss_ld = 0);
 int launch_rmsnorm(const float* x, const void* g, void* out, int rows, int d, float eps,
                    int dtype, cudaStream_t s);
 int launch_rope_table(const BatchDesc& b, float* cos_t, float* sin_t, int head_dim,

@@ -255,6 +255,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int q = 0; q < 8; ++q) res[0][q] = src[q];
       }
+      // fused RMSNorm of the A rows: 1 / rms of this row from the producer's partial sums
+      float rinv = 1.f;
+      if ((EPI == EPI_QKV || EPI == EPI_GELU) && args.ss_in && live) {
+        float ss = 0.f;
+        for (int t2 = 0; t2 < args.ss_n; ++t2) ss += args.ss_in[(size_t)row * args.ss_ld + t2];
+        rinv = rsqrtf(ss / (float)args.norm_d + args.norm_eps);
+      }
       if (!__all_sync(0xffffffffu, PAIR ? mbar_wait_cluster(&acc_full[acc], acc_ph, abort, args.err, 0x104)
                                         : mbar_wait(&acc_full[acc], acc_ph, abort, args.err, 0x104)))
         break;
@@ -284,7 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   const int i = 4 * i4 + e;
-                  const float x = __uint_as_float(ra[i]), y = __uint_as_float(rb[i]);
+                  const float x = __uint_as_float(ra[i]) * rinv, y = __uint_as_float(rb[i]) * rinv;
                   a[i] = x * cv[e] - y * sv[e];
                   b[i] = y * cv[e] + x * sv[e];
                 }
@@ -292,8 +299,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             } else {
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
-                a[i] = __uint_as_float(ra[i]);
-                b[i] = __uint_as_float(rb[i]);
+                a[i] = __uint_as_float(ra[i]) * rinv;
+                b[i] = __uint_as_float(rb[i]) * rinv;
               }
             }
             __nv_bfloat16* dst;
@@ -310,6 +317,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       } else if (EPI == EPI_RESID) {
+        float ssq = 0.f;
         // unrolled so the two residual buffers stay in registers
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
@@ -324,6 +332,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_wait_ld(r);
           if (!live) continue;
           float4* d = reinterpret_cast<float4*>((float*)args.C + (size_t)row * args.ldc + n0 + c * 32);
+          float xs[32];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             float4 x = res[c & 1][q];
@@ -332,8 +341,32 @@ __global__ void __launch_bounds__(THREADS, 1)
             x.z += __uint_as_float(r[4 * q + 2]);
             x.w += __uint_as_float(r[4 * q + 3]);
             d[q] = x;
+            xs[4 * q] = x.x;
+            xs[4 * q + 1] = x.y;
+            xs[4 * q + 2] = x.z;
+            xs[4 * q + 3] = x.w;
+          }
+          if (args.g_next) {
+            // the next RMSNorm's numerator bf16(x g) and this row's sum of squares
+            const uint4* g4 = reinterpret_cast<const uint4*>(args.g_next + n0 + c * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 gu = __ldg(g4 + q);
+              const __nv_bfloat162* gh = reinterpret_cast<const __nv_bfloat162*>(&gu);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 gf = __bfloat1622float2(gh[e]);
+                const int i = 8 * q + 2 * e;
+                ssq = fmaf(xs[i], xs[i], ssq);
+                ssq = fmaf(xs[i + 1], xs[i + 1], ssq);
+                xs[i] *= gf.x;
+                xs[i + 1] *= gf.y;
+              }
+            }
+            store_bf16x32(args.xg + (size_t)row * args.ldc + n0 + c * 32, xs);
           }
         }
+        if (args.g_next && live) args.ss_out[(size_t)row * args.ss_ld + n0 / BN] = ssq;
       } else {
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
@@ -351,7 +384,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           } else {
             if (EPI == EPI_GELU) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+              for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i] * rinv);
             }
             store_bf16x32((__nv_bfloat16*)args.C + (size_t)row * args.ldc + col, v);
           }

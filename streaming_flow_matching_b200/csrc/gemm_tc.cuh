@@ -22,6 +22,19 @@ struct GemmArgs {
   BatchDesc b;
   int block_n;           // N-tile width the B tensor map was built for
   int pair;              // 1: CTA pairs (the B map's box has block_n / 2 rows)
+  // RMSNorm of the updated residual, split across two GEMMs (bf16 path).
+  // EPI_RESID with g_next: also writes xg = bf16(x * g_next) and, per row and
+  // N tile, the partial sum of squares of the updated x: ss_out[row][n0 / BN].
+  const __nv_bfloat16* g_next;
+  __nv_bfloat16* xg;     // [M][N]
+  float* ss_out;         // [M][ss_ld]
+  // EPI_QKV / EPI_GELU with ss_in: A holds bf16(x * g); each accumulator row is
+  // scaled by rsqrt(sum_{t < ss_n} ss_in[row][t] / norm_d + norm_eps).
+  const float* ss_in;    // [M][ss_ld]
+  int ss_n;
+  int ss_ld;
+  int norm_d;
+  float norm_eps;
 };
 
 // Whether an M x N projection runs on CTA pairs (256-row tiles, half of each B

@@ -38,27 +38,37 @@ __device__ __forceinline__ float warp_sum(float v) {
 constexpr int kEmbedRows = 32;
 
 // CL: compile-time bound on c_lat (16, or 64 for any c_lat <= 64), so the
-// W_in row stays in registers.
+// W_in row stays in registers.  With g (bf16 path) the kernel also writes the
+// first RMSNorm's numerator xg = bf16(x g) and, per row and 128-column block,
+// the partial sum of squares ss[row][blockIdx.x] (the QKV GEMM applies 1 / rms).
 template <typename T, int CL>
-__global__ void embed_kernel(const __grid_constant__ BatchDesc b, const __grid_constant__ PtrTable z,
-                             const T* __restrict__ w_in,
-                             const T* __restrict__ e_mod, float tau, float* __restrict__ x, int d,
-                             int c_lat) {
+__global__ void __launch_bounds__(128) embed_kernel(
+    const __grid_constant__ BatchDesc b, const __grid_constant__ PtrTable z,
+    const T* __restrict__ w_in, const T* __restrict__ e_mod, float tau, float* __restrict__ x,
+    int d, int c_lat, const __nv_bfloat16* __restrict__ g, __nv_bfloat16* __restrict__ xg,
+    float* __restrict__ ss, int ss_ld) {
+  __shared__ float red[kEmbedRows][4];
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= d) return;
-  const int half = d / 2;
-  const int ii = i < half ? i : i - half;
-  const double w = pow(10000.0, -2.0 * (double)ii / (double)d);
-  const double ang = 1000.0 * (double)tau * w;
-  const float te = (float)(i < half ? sin(ang) : cos(ang));
-  float wr[CL];
-#pragma unroll
-  for (int c = 0; c < CL; ++c) wr[c] = c < c_lat ? to_f(w_in[(size_t)i * c_lat + c]) : 0.f;
-  const float em_v = to_f(e_mod[i]);
-  const float em_a = to_f(e_mod[d + i]);
+  const bool on = i < d;
   const int rows = b.n * b.n_tok;
   const int r0 = blockIdx.y * kEmbedRows;
-  for (int r = r0; r < r0 + kEmbedRows && r < rows; ++r) {
+  if (!on && !g) return;
+  const int ic = on ? i : 0;
+  const int half = d / 2;
+  const int ii = ic < half ? ic : ic - half;
+  const double w = pow(10000.0, -2.0 * (double)ii / (double)d);
+  const double ang = 1000.0 * (double)tau * w;
+  const float te = (float)(ic < half ? sin(ang) : cos(ang));
+  float wr[CL];
+#pragma unroll
+  for (int c = 0; c < CL; ++c) wr[c] = c < c_lat ? to_f(w_in[(size_t)ic * c_lat + c]) : 0.f;
+  const float em_v = to_f(e_mod[ic]);
+  const float em_a = to_f(e_mod[d + ic]);
+  const float gi = g && on ? __bfloat162float(g[i]) : 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int rr = 0; rr < kEmbedRows; ++rr) {
+    const int r = r0 + rr;
+    if (r >= rows) break;
     const int sess = r / b.n_tok;
     const int j = r - sess * b.n_tok;
     const float* zr = z.p[sess] + (size_t)j * c_lat;
@@ -66,12 +76,26 @@ __global__ void embed_kernel(const __grid_constant__ BatchDesc b, const __grid_c
 #pragma unroll
     for (int c = 0; c < CL; ++c)
       if (c < c_lat) acc = fmaf(zr[c], wr[c], acc);
-    x[(size_t)r * d + i] = acc + (j < b.n_video ? em_v : em_a) + te;
+    const float xv = acc + (j < b.n_video ? em_v : em_a) + te;
+    if (on) x[(size_t)r * d + i] = xv;
+    if (g) {
+      if (on) xg[(size_t)r * d + i] = __float2bfloat16_rn(xv * gi);
+      const float sq = warp_sum(on ? xv * xv : 0.f);
+      if (lane == 0) red[rr][warp] = sq;
+    }
+  }
+  if (g) {
+    __syncthreads();
+    if (threadIdx.x < kEmbedRows && r0 + (int)threadIdx.x < rows) {
+      const float* t = red[threadIdx.x];
+      ss[(size_t)(r0 + threadIdx.x) * ss_ld + blockIdx.x] = (t[0] + t[1]) + (t[2] + t[3]);
+    }
   }
 }
 
 int launch_embed(const BatchDesc& b, float* const* z, const void* w_in, const void* e_mod,
-                 float tau, float* x, int d, int c_lat, int dtype, cudaStream_t s) {
+                 float tau, float* x, int d, int c_lat, int dtype, cudaStream_t s,
+                 const void* g, void* xg, float* ss, int ss_ld) {
   PtrTable t{};
   for (int i = 0; i < b.n; ++i) t.p[i] = z[i];
   const int rows = b.n * b.n_tok;
@@ -81,10 +105,12 @@ int launch_embed(const BatchDesc& b, float* const* z, const void* w_in, const vo
   if (dtype == SFM_DTYPE_BF16) {
     auto k = c16 ? embed_kernel<__nv_bfloat16, 16> : embed_kernel<__nv_bfloat16, 64>;
     k<<<grid, 128, 0, s>>>(b, t, (const __nv_bfloat16*)w_in, (const __nv_bfloat16*)e_mod, tau, x,
-                           d, c_lat);
+                           d, c_lat, (const __nv_bfloat16*)g, (__nv_bfloat16*)xg, ss, ss_ld);
   } else {
+    if (g) return SFM_EINVAL;    // the fused norm is a bf16-path feature
     auto k = c16 ? embed_kernel<float, 16> : embed_kernel<float, 64>;
-    k<<<grid, 128, 0, s>>>(b, t, (const float*)w_in, (const float*)e_mod, tau, x, d, c_lat);
+    k<<<grid, 128, 0, s>>>(b, t, (const float*)w_in, (const float*)e_mod, tau, x, d, c_lat, nullptr,
+                           nullptr, nullptr, 0);
   }
   return record_cuda(cudaGetLastError());
 }

@@ -76,6 +76,38 @@ def test_velocity_and_solve_match_oracle(cuda_device, w):
     p.close()
 
 
+def test_velocity_with_random_norm_gains_matches_oracle(cuda_device):
+    # the synthetic weights have unit RMSNorm gains; here every gain vector (both norms
+    # of every layer and the final one) is drawn from U[0.5, 1.5], so each gain must be
+    # applied at its own norm, including in the bf16 path where the norm is split
+    # between the kernel that updates x and the next projection
+    w = SMALL_BF16
+    weights_cpu = S.make_weights(w)
+    g = torch.Generator().manual_seed(31)
+    def draw(t):
+        return (0.5 + torch.rand(t.shape, generator=g)).to(t.dtype)
+    weights_cpu["g_final"] = draw(weights_cpu["g_final"])
+    for lay in weights_cpu["layers"]:
+        lay["g_attn"] = draw(lay["g_attn"])
+        lay["g_mlp"] = draw(lay["g_mlp"])
+    weights = to_cuda(weights_cpu)
+    k, v = S.make_kv_slices(w, w.cache_units)
+    p = _performer(w, weights)
+    s = p.open_session(w.cache_units)
+    p.kvcache_append(s, k.cuda(), v.cuda())
+    _, eps = S.make_latents(w)
+    eps = eps[0]
+    z = eps.cuda().clone()
+    vel = torch.empty_like(z)
+    p.denoise_step(s, z, 1.0, 0.75, vel)
+    torch.cuda.synchronize()
+    ref_v = _oracle_velocity(w, weights_cpu, k, v, w.cache_units, eps, 1.0)
+    e_v = rel_l2(vel.cpu().numpy(), ref_v)
+    print(f"random gains: velocity {e_v:.3e}")
+    assert e_v <= BF16_TOL, e_v
+    p.close()
+
+
 def test_ring_wrapped_cache_velocity_matches_oracle(cuda_device):
     # 7 units into 5 slots: units 5, 6 overwrite slots 0, 1; positions keep counting
     w = SMALL_BF16

@@ -1,6 +1,8 @@
 // Blackwell (sm_100a) building blocks: mbarriers with bounded waits, TMA tile
-// loads (no multicast), tensor memory (TMEM) allocation / loads / stores, and
-// the shared-memory and instruction descriptors of tcgen05.mma (kind::f16).
+// loads (no multicast), tensor memory (TMEM) allocation / loads / stores, the
+// shared-memory and instruction descriptors of tcgen05.mma (kind::f16), and the
+// CTA-pair (cluster of two, cta_group::2) forms of allocation, MMA, commit and
+// TMA completion used by the GEMM.
 //
 // Every wait is bounded: after kWaitNs nanoseconds a waiter raises the CTA's
 // abort flag and the kernel's global error word, and the roles of the kernel
@@ -164,9 +166,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[15])
       : "memory");
 }
-__device__ __forceinline__ void tmem_ld_wait() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 // Waits for this thread's outstanding tcgen05.ld and ties the destination
 // registers to the wait, so no use of them can be scheduled before it.
 __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
@@ -272,9 +271,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;

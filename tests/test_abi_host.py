@@ -67,6 +67,7 @@ def test_null_arguments_are_rejected():
     assert L.lib.sfm_euler_update(None, None, 0.5, 0, None) == L.SFM_OK   # empty is a no-op
     assert L.lib.sfm_attention(None, None, None, None, 4, 4, 1, 128, 0, None, 0, None) == L.SFM_EINVAL
     assert L.lib.sfm_attention_workspace_bytes(924, 58524, 24, 128, L.SFM_DTYPE_FP32) == 0
+    assert L.lib.sfm_set_graph_mode(None, 1) == L.SFM_EINVAL
     assert L.lib.sfm_strerror(L.SFM_ESESSION) == b"unknown or closed session"
     assert L.lib.sfm_strerror(12345) == b"unknown status"
 

@@ -6,7 +6,7 @@
 
 namespace sfm {
 
-constexpr int kMaxSplits = 8;
+constexpr int kMaxSplits = 16;
 // TMA box heights of the tcgen05 attention kernel: query and key / value tiles
 // of 128 rows (one 64-dim half of a head per box).
 constexpr int kAttnQBoxRows = 128;

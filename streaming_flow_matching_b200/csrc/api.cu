@@ -60,6 +60,8 @@ struct sfm_handle {
   std::vector<CUtensorMap> map_wqkv, map_wo, map_w1, map_w2;
   int bn_qkv = 0, bn_o = 0, bn_up = 0, bn_down = 0;   // N-tile widths the weight maps use
   bool pair_qkv = false, pair_o = false, pair_up = false, pair_down = false;   // CTA pairs
+  int ksplit_o = 1, ksplit_down = 1;     // K slices of the residual projections (few tiles)
+  float* ws_splitk = nullptr;            // [slices][M][d] fp32 partials
   std::vector<void*> owned;
 
   void* layer_k(int l) const { return (char*)k_pool + (size_t)l * cfg.pool_tokens * hd * es; }
@@ -215,6 +217,18 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
     g.norm_eps = eps;
     return g;
   };
+  // a residual projection in K slices: fp32 partials, then x += their sum (and the
+  // next norm's numerator and the row's whole sum of squares)
+  auto resid_split = [&](const CUtensorMap& ma, const CUtensorMap& mb, int K, int bn, int slices,
+                         const void* gain) {
+    GemmArgs g = gemm_args(M, d, K, EPI_F32, h->ws_splitk, d, h->d_err, bn, false);
+    g.k_splits = slices;
+    int r = launch_gemm_tc(ma, mb, g, h->sms, s);
+    if (!r)
+      r = launch_resid_splitk(h->x, h->ws_splitk, slices, M, d, gain, h->xn, h->ss, ss_ld, s);
+    if (gain) ss_n = 1;
+    return r;
+  };
   auto norm_next = [&](GemmArgs g, const void* gain, int bn) {   // a producer
     if (!gain) return g;
     g.g_next = (const __nv_bfloat16*)gain;
@@ -265,7 +279,9 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
     }
     {
       ProfScope ps(SFM_PROF_GEMM_O, s);
-      if (tc) {
+      if (tc && h->ksplit_o > 1) {
+        SFM_TRY(resid_split(h->map_ao, h->map_wo[l], hd, h->bn_o, h->ksplit_o, h->g_mlp[l]));
+      } else if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_ao, h->map_wo[l],
                                norm_next(gemm_args(M, d, hd, EPI_RESID, h->x, d, h->d_err, h->bn_o, h->pair_o),
                                          h->g_mlp[l], h->bn_o),
@@ -290,7 +306,10 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
     }
     {
       ProfScope ps(SFM_PROF_GEMM_DOWN, s);
-      if (tc) {
+      if (tc && h->ksplit_down > 1) {
+        SFM_TRY(resid_split(h->map_hmlp, h->map_w2[l], F, h->bn_down, h->ksplit_down,
+                            l + 1 < c.n_layers ? h->g_attn[l + 1] : nullptr));
+      } else if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_hmlp, h->map_w2[l],
                                norm_next(gemm_args(M, d, F, EPI_RESID, h->x, d, h->d_err, h->bn_down, h->pair_down),
                                          l + 1 < c.n_layers ? h->g_attn[l + 1] : nullptr, h->bn_down),
@@ -492,6 +511,13 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     h->bn_up = gemm_tc_block_n(mm, F_, 0, EPI_GELU, h->sms, h->pair_up);
     h->bn_down = gemm_tc_block_n(mm, d_, 0, EPI_RESID, h->sms, h->pair_down);
     if (!h->bn_qkv || !h->bn_o || !h->bn_up || !h->bn_down) rc = SFM_EUNSUPPORTED;
+    if (!rc) {
+      // split-K for residual projections whose tiles fill under half of the SMs
+      if (!h->pair_o) h->ksplit_o = gemm_tc_k_splits(mm, d_, hd_, h->bn_o, h->sms);
+      if (!h->pair_down) h->ksplit_down = gemm_tc_k_splits(mm, d_, F_, h->bn_down, h->sms);
+      const int ks = h->ksplit_o > h->ksplit_down ? h->ksplit_o : h->ksplit_down;
+      if (ks > 1) rc = dalloc(h, &h->ws_splitk, (size_t)ks * M * d_ * 4);
+    }
     // the B box holds the weight rows one CTA stages: half the tile on pairs
     for (int l = 0; l < L_ && !rc; ++l) {
       rc = make_b_map(&h->map_wqkv[l], h->w_qkv[l], 3 * hd_, d_, h->bn_qkv / (h->pair_qkv ? 2 : 1));

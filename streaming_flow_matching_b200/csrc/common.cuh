@@ -65,6 +65,11 @@ int launch_kv_read(const void* k_pool, const void* v_pool, void* k_dst, void* v_
 
 // With g (bf16 only): also xg = bf16(x g) and per-row partial sums of squares
 // over 128-column blocks into ss ([rows][ss_ld]) -- the first RMSNorm, fused.
+// Second half of a split-K residual projection (bf16 path): x += sum of the
+// slices' partials ws[s][rows][d]; with g_next (bf16) also xg = bf16(x g) and
+// the row's sum of squares into ss[row * ss_ld].
+int launch_resid_splitk(float* x, const float* ws, int n_slices, int rows, int d,
+                        const void* g_next, void* xg, float* ss, int ss_ld, cudaStream_t s);
 int launch_embed(const BatchDesc& b, float* const* z, const void* w_in, const void* e_mod,
                  float tau, float* x, int d, int c_lat, int dtype, cudaStream_t s,
                  const void* g = nullptr, void* xg = nullptr, float* ss = nullptr, int ss_ld = 0);

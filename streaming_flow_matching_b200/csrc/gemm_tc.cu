@@ -93,6 +93,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int n_tiles = args.N / BN;
   const int tiles = m_tiles * n_tiles;
   const int kblocks = args.K / BK;
+  const int ksp = args.k_splits > 1 ? args.k_splits : 1;
+  const int units_total = tiles * ksp;       // (tile, k slice) work units
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -138,10 +140,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       int last_parity[8];
       for (int i = 0; i < C::STAGES; ++i) last_parity[i] = -1;
       bool ok = true;
-      for (int t = unit; t < tiles && ok; t += n_units) {
+      for (int u = unit; u < units_total && ok; u += n_units) {
+        const int t = u % tiles, sl = u / tiles;
         const int m0 = (t % m_tiles) * TM + (int)rank * BM;
         const int n0 = (t / m_tiles) * BN + (int)rank * C::B_ROWS;
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = sl * kblocks / ksp; kb < (sl + 1) * kblocks / ksp; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, abort, args.err, 0x101)) {
             ok = false;
             break;
@@ -186,7 +189,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       int acc = 0;
       uint32_t acc_ph = 0;
       bool ok = true, issued = false;
-      for (int t = unit; t < tiles && ok; t += n_units) {
+      for (int u = unit; u < units_total && ok; u += n_units) {
+        const int sl = u / tiles;
+        const int kb0 = sl * kblocks / ksp, kb1 = (sl + 1) * kblocks / ksp;
         if (!(PAIR ? mbar_wait_cluster(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102)
                    : mbar_wait(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102))) {
           ok = false;
@@ -194,7 +199,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * C::ACC_COLS);
-        for (int kb = 0; kb < kblocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[s], ph, abort, args.err, 0x103)) {
             ok = false;
             break;
@@ -207,10 +212,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int k = 0; k < BK / 16; ++k) {  // +32 bytes per K=16 step inside the swizzle atom
             if (PAIR)
               umma_bf16_pair(d, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
-                             (kb | k) != 0 ? 1u : 0u);
+                             (kb != kb0 || k != 0) ? 1u : 0u);
             else
               umma_bf16(d, da + (uint64_t)(2 * k), db + (uint64_t)(2 * k), idesc,
-                        (kb | k) != 0 ? 1u : 0u);
+                        (kb != kb0 || k != 0) ? 1u : 0u);
           }
           issued = true;
           if (PAIR)
@@ -243,7 +248,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;              // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_ph = 0;
-    for (int t = unit; t < tiles; t += n_units) {
+    for (int u = unit; u < units_total; u += n_units) {
+      const int t = u % tiles, sl = u / tiles;
       const int m0 = (t % m_tiles) * TM + (int)rank * BM, n0 = (t / m_tiles) * BN;
       const int row = m0 + quarter * 32 + lane;
       const bool live = row < args.M;
@@ -378,7 +384,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
           const int col = n0 + c * 32;
           if (EPI == EPI_F32) {
-            float4* d = reinterpret_cast<float4*>((float*)args.C + (size_t)row * args.ldc + col);
+            float4* d = reinterpret_cast<float4*>((float*)args.C + (size_t)sl * args.M * args.ldc +
+                                                  (size_t)row * args.ldc + col);
 #pragma unroll
             for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
           } else {
@@ -426,7 +433,7 @@ int launch_bn(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, 
               cudaStream_t s) {
   using C = Cfg<BN, PAIR>;
   constexpr int TM = PAIR ? 2 * BM : BM;
-  const int tiles = ((args.M + TM - 1) / TM) * (args.N / BN);
+  const int tiles = ((args.M + TM - 1) / TM) * (args.N / BN) * (args.k_splits > 1 ? args.k_splits : 1);
   const int units = PAIR ? sms / 2 : sms;
   const int grid = (tiles < units ? tiles : units) * (PAIR ? 2 : 1);
   auto kern = gemm_tc_kernel<BN, EPI, PAIR>;
@@ -483,6 +490,17 @@ int gemm_tc_block_n(int M, int N, int hd, int epi, int sms, bool pair) {
   return best;
 }
 
+int gemm_tc_k_splits(int M, int N, int K, int block_n, int sms) {
+  if (block_n <= 0 || N % block_n) return 1;
+  const long long tiles = (long long)((M + gtc::BM - 1) / gtc::BM) * (N / block_n);
+  if (2 * tiles > sms) return 1;
+  long long sp = sms / tiles;
+  const long long by_k = (K / gtc::BK) / 4;   // at least 4 k-blocks per slice
+  if (sp > by_k) sp = by_k;
+  if (sp > 16) sp = 16;
+  return sp > 1 ? (int)sp : 1;
+}
+
 int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,
                    cudaStream_t s) {
   if (args.M <= 0) return SFM_OK;
@@ -491,6 +509,8 @@ int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& a
   const int bn = args.block_n;
   if (!bn || args.N % bn || args.K % gtc::BK || args.K <= 0) return SFM_EUNSUPPORTED;
   if (args.epi == EPI_QKV && (args.hd % bn || args.N != 3 * args.hd)) return SFM_EUNSUPPORTED;
+  if (args.k_splits > 1 && (args.epi != EPI_F32 || pair || args.k_splits > args.K / gtc::BK))
+    return SFM_EUNSUPPORTED;
 #define SFM_GTC(BN_, E)                                                              \
   if (bn == BN_ && args.epi == E)                                                    \
     return pair ? gtc::launch_bn<BN_, E, true>(a, b, args, sms, s)                  \

@@ -35,6 +35,9 @@ struct GemmArgs {
   int ss_ld;
   int norm_d;
   float norm_eps;
+  // split-K (EPI_F32 only): unit u covers tile u % tiles and k-blocks of slice
+  // u / tiles; slice s writes its fp32 partial to C + s * M * ldc
+  int k_splits;          // 0 or 1: no split
 };
 
 // Whether an M x N projection runs on CTA pairs (256-row tiles, half of each B
@@ -43,6 +46,9 @@ bool gemm_tc_pair(int M, int N, int hd, int epi, int sms);
 // N-tile width (256, 192 or 128) for an M x N problem on `sms` SMs, in the given
 // mode; 0 if none fits.
 int gemm_tc_block_n(int M, int N, int hd, int epi, int sms, bool pair);
+// K slices for a projection whose tiles fill under half of the SMs (single-CTA
+// mode, at least 4 k-blocks per slice); 1 when no split pays.
+int gemm_tc_k_splits(int M, int N, int K, int block_n, int sms);
 // A: tensor map over [M_alloc][K] bf16, box {64, 128}; B: over [N][K], box
 // {64, pair ? block_n / 2 : block_n}.
 int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args, int sms,

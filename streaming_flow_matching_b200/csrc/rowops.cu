@@ -183,6 +183,63 @@ __global__ void __launch_bounds__(1024) rmsnorm_kernel(const float* __restrict__
   store8(out + (size_t)row * d + c, v);
 }
 
+// Split-K residual projection, second half: x += the K slices' partial
+// products (ws[s][row][:], summed in slice order), and with g_next the next
+// RMSNorm's numerator bf16(x g) and the row's sum of squares ss[row][0].
+// One CTA per row, 8 columns per thread.
+__global__ void __launch_bounds__(1024) resid_splitk_kernel(
+    float* __restrict__ x, const float* __restrict__ ws, int n_slices, int rows, int d,
+    const __nv_bfloat16* __restrict__ g_next, __nv_bfloat16* __restrict__ xg,
+    float* __restrict__ ss, int ss_ld) {
+  __shared__ float red[32];
+  const int row = blockIdx.x;
+  const int c = threadIdx.x * 8;
+  const bool on = c < d;
+  float v[8];
+  float sq = 0.f;
+  if (on) {
+    load8(x + (size_t)row * d + c, v);
+    for (int sl = 0; sl < n_slices; ++sl) {
+      float p[8];
+      load8(ws + ((size_t)sl * rows + row) * d + c, p);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] += p[i];
+    }
+    store8(x + (size_t)row * d + c, v);
+    if (g_next) {
+      float gv[8];
+      load8(g_next + c, gv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        sq = fmaf(v[i], v[i], sq);
+        v[i] *= gv[i];
+      }
+      store8(xg + (size_t)row * d + c, v);
+    }
+  }
+  if (!g_next) return;
+  sq = warp_sum(sq);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = sq;
+  __syncthreads();
+  if (warp == 0) {
+    float t = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.f;
+    t = warp_sum(t);
+    if (lane == 0) ss[(size_t)row * ss_ld] = t;
+  }
+}
+
+int launch_resid_splitk(float* x, const float* ws, int n_slices, int rows, int d,
+                        const void* g_next, void* xg, float* ss, int ss_ld, cudaStream_t s) {
+  if (rows <= 0) return SFM_OK;
+  if (d % 8 || d / 8 > 1024) return SFM_EUNSUPPORTED;
+  const int threads = ((d / 8) + 31) / 32 * 32;
+  resid_splitk_kernel<<<rows, threads, 0, s>>>(x, ws, n_slices, rows, d,
+                                              (const __nv_bfloat16*)g_next, (__nv_bfloat16*)xg,
+                                              ss, ss_ld);
+  return record_cuda(cudaGetLastError());
+}
+
 int launch_rmsnorm(const float* x, const void* g, void* out, int rows, int d, float eps,
                    int dtype, cudaStream_t s) {
   if (rows <= 0) return SFM_OK;

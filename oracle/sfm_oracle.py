@@ -328,6 +328,41 @@ def denoise_solve(cfg: Config, eps, taus, w, cache_k, cache_v, valid_tokens, p0)
 
 
 # ---------------------------------------------------------------------------
+# classifier-free guidance (the distillation teacher's sampler)
+# ---------------------------------------------------------------------------
+
+def guided_velocity(v_cond, v_uncond, scale):
+    """Classifier-free guidance: start from the unconditional velocity and move
+    `scale` times the conditional-minus-unconditional difference.
+
+    [v0.1] training, Stage 3 (low-latency distillation): the teacher samples with
+    classifier-free guidance and more solver steps; the pages give no formula.
+    Reading: the usual form of Ho & Salimans (2022), v_u + s (v_c - v_u), so
+    s = 1 is the conditional model and s = 0 the unconditional one.
+    """
+    v_u = f64(v_uncond)
+    return v_u + float(scale) * (f64(v_cond) - v_u)
+
+
+def denoise_solve_cfg(cfg: Config, eps, taus, w, cond, uncond, scale):
+    """Guided solve of one unit: at every Euler step f_theta is evaluated twice at
+    the same z and tau, once on the conditional context and once on the
+    unconditional one, and the step follows their guided velocity.
+
+    cond / uncond: (cache_k, cache_v, valid_tokens, p0) of the two contexts.  The
+    performer's only condition is the thinker's K/V in its cache ([abs]: the
+    thinker reaches the performer only as K/V conditioning), so the
+    unconditional context is a cache holding a null condition; an empty cache
+    (valid_tokens = 0: the unit attends to itself alone) is the plainest one.
+    """
+    def velocity(z, t):
+        v_c = f_theta(cfg, z, t, w, *cond)
+        v_u = f_theta(cfg, z, t, w, *uncond)
+        return guided_velocity(v_c, v_u, scale)
+    return fm_solve(eps, taus, velocity)
+
+
+# ---------------------------------------------------------------------------
 # block-causal full-sequence form (prefill / invariant checks)
 # ---------------------------------------------------------------------------
 

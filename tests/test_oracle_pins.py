@@ -374,3 +374,61 @@ def test_step_flops_counts():
     attn = 4 * 924 * (57600 + 924) * 3072
     assert abs(attn / 28 / 1e9 * 28 - attn / 1e9) < 1e-9
     assert abs(f / 1e12 - 24.47) < 0.01          # per Euler step at the 640x368 unit
+
+
+# --------------------------------------------------------------------------
+# classifier-free guidance
+# --------------------------------------------------------------------------
+
+def test_guided_velocity_closed_form_with_exact_fields():
+    # Constant fields aiming at two clean latents a (conditional) and b
+    # (unconditional): one Euler step 1 -> 0 from eps lands on b + s (a - b), so
+    # s = 0, 1 give b and a, and s = 3 extrapolates three times past b.
+    rng = np.random.default_rng(40)
+    a, b, eps = (rng.standard_normal((5, 3)) for _ in range(3))
+    for s in (0.0, 1.0, 3.0, -0.5):
+        v = O.guided_velocity(O.rf_velocity(a, eps), O.rf_velocity(b, eps), s)
+        got = O.fm_solve(eps, [1.0, 0.0], lambda z, t, v=v: v)
+        np.testing.assert_allclose(got, b + s * (a - b), rtol=0, atol=1e-14)
+
+
+def _cfg_problem(seed):
+    cfg, w, ck, cv, z, S = _tiny_problem(seed)
+    rng = np.random.default_rng(seed + 100)
+    uk = [rng.standard_normal(c.shape) for c in ck]
+    uv = [rng.standard_normal(c.shape) for c in cv]
+    return cfg, w, z, (ck, cv, S, 7), (uk, uv, 2, 0)
+
+
+def test_guided_solve_scale_one_is_conditional_and_zero_is_unconditional():
+    cfg, w, z, cond, uncond = _cfg_problem(41)
+    taus = [1.0, 0.6, 0.2, 0.0]
+    c = O.denoise_solve(cfg, z, taus, w, *cond)
+    u = O.denoise_solve(cfg, z, taus, w, *uncond)
+    assert np.max(np.abs(c - u)) > 1e-3                 # the two contexts differ
+    np.testing.assert_allclose(O.denoise_solve_cfg(cfg, z, taus, w, cond, uncond, 1.0), c,
+                               rtol=0, atol=1e-12)
+    np.testing.assert_allclose(O.denoise_solve_cfg(cfg, z, taus, w, cond, uncond, 0.0), u,
+                               rtol=0, atol=1e-12)
+
+
+def test_guided_solve_with_equal_contexts_ignores_the_scale():
+    cfg, w, z, cond, _ = _cfg_problem(42)
+    taus = [1.0, 0.5, 0.0]
+    plain = O.denoise_solve(cfg, z, taus, w, *cond)
+    for s in (0.0, 2.5, 7.0):
+        np.testing.assert_allclose(O.denoise_solve_cfg(cfg, z, taus, w, cond, cond, s), plain,
+                                   rtol=0, atol=1e-11)
+
+
+def test_guided_solve_matches_brute_force_velocities():
+    # Two Euler steps with the scalar-loop velocity network on each context.
+    cfg, w, z, cond, uncond = _cfg_problem(43)
+    s = 4.0
+    got = O.denoise_solve_cfg(cfg, z, [1.0, 0.5, 0.0], w, cond, uncond, s)
+    zz = z
+    for t in (1.0, 0.5):
+        vc = np.array(BF.velocity(cfg, zz, t, w, *cond))
+        vu = np.array(BF.velocity(cfg, zz, t, w, *uncond))
+        zz = zz - 0.5 * (vu + s * (vc - vu))
+    np.testing.assert_allclose(got, zz, rtol=1e-10, atol=1e-11)

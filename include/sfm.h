@@ -185,6 +185,42 @@ SFM_API int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessi
                          float* const* z, const float* taus, int n_taus, void* stream);
 
 /*
+ * Classifier-free-guided solve, the sampler of the distillation teacher
+ * ("Wan-Streamer" v0.1 blog, training, Stage 3: classifier-free guidance and
+ * more flow-matching solver steps).  At every Euler step f_theta runs twice at
+ * the same z and tau -- on `session` (the conditional context: the thinker's
+ * K/V in its cache) and on `uncond_session` (the unconditional context) -- and
+ * the step follows the guided velocity v = v_u + scale * (v_c - v_u), so
+ * scale = 1 is the plain conditional solve and scale = 0 the unconditional
+ * one.  The pages give no formula; this is the usual form of classifier-free
+ * guidance.  The unconditional context is whatever uncond_session's cache
+ * holds: a session with nothing appended (the unit attends to itself alone)
+ * drops the condition entirely; one holding the K/V of a null prompt is the
+ * other common choice.
+ *   - z: device fp32 [N][C], updated in place (the one latent both
+ *     evaluations read).  taus as for sfm_fm_solve.  Both evaluations write
+ *     their unit's K/V into their own session's scratch rows, as a plain
+ *     solve does; neither cache's contents or unit count change.
+ *   - SFM_EINVAL if the two sessions are the same or scale is not finite.
+ *   - Runs as one batch of two evaluations: needs max_sessions >= 2
+ *     (SFM_ECAPACITY otherwise).
+ */
+SFM_API int sfm_fm_solve_guided(sfm_handle* h, int session, int uncond_session, float* z,
+                                const float* taus, int n_taus, float scale, void* stream);
+/*
+ * n_pairs guided solves in one batch of 2 * n_pairs evaluations.  sessions,
+ * uncond_sessions, z: host arrays of n_pairs entries (z[p] device fp32
+ * [N][C]); all 2 * n_pairs session ids distinct.  v_out: NULL, or a host
+ * array of n_pairs device fp32 [N][C] buffers (entries may be NULL) that
+ * receive the guided velocity of the last step.  SFM_ECAPACITY if
+ * 2 * n_pairs > max_sessions.
+ */
+SFM_API int sfm_fm_solve_guided_batched(sfm_handle* h, int n_pairs, const int* sessions,
+                                        const int* uncond_sessions, float* const* z,
+                                        const float* taus, int n_taus, float scale,
+                                        float* const* v_out, void* stream);
+
+/*
  * Launch mode of sfm_denoise_step / sfm_fm_solve / sfm_fm_solve_batched.
  * enabled = 1 (the default): each call is captured into one CUDA graph on a
  * stream private to the handle and the graph is launched on the caller's

@@ -67,6 +67,9 @@ def _load():
         "sfm_denoise_step": (i, [vp, i, vp, f, f, vp, vp]),
         "sfm_fm_solve": (i, [vp, i, vp, C.POINTER(f), i, vp]),
         "sfm_fm_solve_batched": (i, [vp, i, C.POINTER(i), C.POINTER(vp), C.POINTER(f), i, vp]),
+        "sfm_fm_solve_guided": (i, [vp, i, i, vp, C.POINTER(f), i, f, vp]),
+        "sfm_fm_solve_guided_batched": (i, [vp, i, C.POINTER(i), C.POINTER(i), C.POINTER(vp),
+                                            C.POINTER(f), i, f, C.POINTER(vp), vp]),
         "sfm_set_graph_mode": (i, [vp, i]),
         "sfm_attention_workspace_bytes": (sz, [i, i, i, i, i]),
         "sfm_attention": (i, [vp, vp, vp, vp, i, i, i, i, i, vp, sz, vp]),
@@ -93,7 +96,8 @@ lib = _load()
 # Every symbol declared in include/sfm.h, in declaration order.
 EXPORTS = ["sfm_create", "sfm_destroy", "sfm_session_open", "sfm_session_reset",
            "sfm_session_get_info", "sfm_kvcache_append", "sfm_kvcache_read", "sfm_denoise_step",
-           "sfm_fm_solve", "sfm_fm_solve_batched", "sfm_set_graph_mode", "sfm_attention_workspace_bytes",
+           "sfm_fm_solve", "sfm_fm_solve_batched", "sfm_fm_solve_guided",
+           "sfm_fm_solve_guided_batched", "sfm_set_graph_mode", "sfm_attention_workspace_bytes",
            "sfm_attention", "sfm_attention_noalloc", "sfm_linear", "sfm_euler_update", "sfm_profile_begin", "sfm_profile_end",
            "sfm_kernel_launch_count", "sfm_check_device_error", "sfm_strerror",
            "sfm_last_cuda_error"]

@@ -37,7 +37,7 @@ struct sfm_handle {
   // solves run as one CUDA graph, captured on a private stream and updated in place
   bool graphs = true;
   cudaStream_t cap_stream = nullptr;
-  cudaGraphExec_t graph_exec = nullptr;
+  cudaGraphExec_t graph_exec[2] = {nullptr, nullptr};   // plain / guided solves
   long long pool_used = 0;
   std::vector<Session> sessions;
   // scratch, sized for max_sessions * n_tok rows
@@ -183,9 +183,15 @@ GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err, int
   return g;
 }
 
+struct Guidance {
+  bool on = false;
+  float scale = 1.f;
+};
+
 // One Euler step of f_theta for the sessions in b (RoPE table already filled).
+// Guided: entries 2p, 2p + 1 are a conditional / unconditional pair sharing z[2p].
 int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from, float tau_to,
-             float* const* v_out, cudaStream_t s) {
+             float* const* v_out, const Guidance& gd, cudaStream_t s) {
   const sfm_config& c = h->cfg;
   const int M = b.n * b.n_tok;
   const int d = c.d_model, hd = h->hd, F = c.d_mlp, dt = c.dtype;
@@ -322,7 +328,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
   {
     ProfScope ps(SFM_PROF_HEAD, s);
     SFM_TRY(launch_head_euler(b, h->x, h->g_final, h->w_out, z, v_out, tau_to - tau_from, d,
-                              c.c_lat, eps, dt, s));
+                              c.c_lat, eps, dt, s, gd.on, gd.scale));
   }
 #undef SFM_TRY
   return SFM_OK;
@@ -336,7 +342,7 @@ int check_taus(const float* taus, int n_taus) {
 }
 
 int solve_direct(sfm_handle* h, int n, const int* sessions, float* const* z, const float* taus,
-                 int n_taus, float* const* v_out, cudaStream_t s) {
+                 int n_taus, float* const* v_out, const Guidance& gd, cudaStream_t s) {
   BatchDesc b;
   fill_batch(h, n, sessions, &b);
   int rc;
@@ -346,7 +352,7 @@ int solve_direct(sfm_handle* h, int n, const int* sessions, float* const* z, con
   }
   if (rc) return rc;
   for (int i = 0; i + 1 < n_taus; ++i) {
-    rc = run_step(h, b, z, taus[i], taus[i + 1], v_out, s);
+    rc = run_step(h, b, z, taus[i], taus[i + 1], v_out, gd, s);
     if (rc) return rc;
   }
   return SFM_OK;
@@ -360,12 +366,13 @@ int solve_direct(sfm_handle* h, int n, const int* sessions, float* const* z, con
 // nor per-launch overheads.  The profiler brackets every launch with events,
 // so a profiled call launches directly.
 int solve(sfm_handle* h, int n, const int* sessions, float* const* z, const float* taus,
-          int n_taus, float* const* v_out, cudaStream_t s) {
+          int n_taus, float* const* v_out, cudaStream_t s, const Guidance& gd = Guidance{}) {
   if (!h->graphs || !h->cap_stream || profiling_active())
-    return solve_direct(h, n, sessions, z, taus, n_taus, v_out, s);
+    return solve_direct(h, n, sessions, z, taus, n_taus, v_out, gd, s);
+  cudaGraphExec_t& exec = h->graph_exec[gd.on ? 1 : 0];
   if (cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
     return record_cuda(cudaGetLastError());
-  const int rc = solve_direct(h, n, sessions, z, taus, n_taus, v_out, h->cap_stream);
+  const int rc = solve_direct(h, n, sessions, z, taus, n_taus, v_out, gd, h->cap_stream);
   cudaGraph_t g = nullptr;
   const cudaError_t ec = cudaStreamEndCapture(h->cap_stream, &g);
   if (rc || ec != cudaSuccess || !g) {
@@ -373,22 +380,22 @@ int solve(sfm_handle* h, int n, const int* sessions, float* const* z, const floa
     cudaGetLastError();
     return rc ? rc : record_cuda(ec != cudaSuccess ? ec : cudaErrorStreamCaptureInvalidated);
   }
-  if (h->graph_exec) {
+  if (exec) {
     cudaGraphExecUpdateResultInfo info;
-    if (cudaGraphExecUpdate(h->graph_exec, g, &info) != cudaSuccess) {
+    if (cudaGraphExecUpdate(exec, g, &info) != cudaSuccess) {
       cudaGetLastError();
-      cudaGraphExecDestroy(h->graph_exec);
-      h->graph_exec = nullptr;
+      cudaGraphExecDestroy(exec);
+      exec = nullptr;
     }
   }
   cudaError_t e = cudaSuccess;
-  if (!h->graph_exec) e = cudaGraphInstantiate(&h->graph_exec, g, 0);
+  if (!exec) e = cudaGraphInstantiate(&exec, g, 0);
   cudaGraphDestroy(g);
   if (e != cudaSuccess) {
-    h->graph_exec = nullptr;
+    exec = nullptr;
     return record_cuda(e);
   }
-  return record_cuda(cudaGraphLaunch(h->graph_exec, s));
+  return record_cuda(cudaGraphLaunch(exec, s));
 }
 
 }  // namespace
@@ -537,7 +544,8 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
 void sfm_destroy(sfm_handle* h) {
   if (!h) return;
   cudaDeviceSynchronize();
-  if (h->graph_exec) cudaGraphExecDestroy(h->graph_exec);
+  for (cudaGraphExec_t e : h->graph_exec)
+    if (e) cudaGraphExecDestroy(e);
   if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   for (void* p : h->owned) cudaFree(p);
   delete h;
@@ -639,11 +647,13 @@ int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long long row0
 int sfm_set_graph_mode(sfm_handle* h, int enabled) {
   if (!h || (enabled != 0 && enabled != 1)) return SFM_EINVAL;
   h->graphs = enabled != 0;
-  if (!h->graphs && h->graph_exec) {
-    // launches already enqueued keep their copy of the graph
-    cudaGraphExecDestroy(h->graph_exec);
-    h->graph_exec = nullptr;
-  }
+  if (!h->graphs)
+    for (cudaGraphExec_t& e : h->graph_exec)
+      if (e) {
+        // launches already enqueued keep their copy of the graph
+        cudaGraphExecDestroy(e);
+        e = nullptr;
+      }
   return SFM_OK;
 }
 
@@ -682,6 +692,43 @@ int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions, flo
   }
   if ((rc = check_taus(taus, n_taus))) return rc;
   return solve(h, n_sessions, sessions, z, taus, n_taus, nullptr, (cudaStream_t)stream);
+}
+
+int sfm_fm_solve_guided_batched(sfm_handle* h, int n_pairs, const int* sessions,
+                                const int* uncond_sessions, float* const* z, const float* taus,
+                                int n_taus, float scale, float* const* v_out, void* stream) {
+  if (!h || !sessions || !uncond_sessions || !z || n_pairs < 1) return SFM_EINVAL;
+  if (!h->has_weights || !isfinite(scale)) return SFM_EINVAL;
+  if (n_pairs > kMaxBatch / 2 || 2 * n_pairs > h->cfg.max_sessions) return SFM_ECAPACITY;
+  int rc;
+  int ids[kMaxBatch];
+  float* zs[kMaxBatch];
+  float* vs[kMaxBatch];
+  for (int p = 0; p < n_pairs; ++p) {
+    if (!z[p]) return SFM_EINVAL;
+    ids[2 * p] = sessions[p];
+    ids[2 * p + 1] = uncond_sessions[p];
+    zs[2 * p] = zs[2 * p + 1] = z[p];
+    vs[2 * p] = vs[2 * p + 1] = v_out ? v_out[p] : nullptr;
+  }
+  // every session (conditional or not) distinct: each evaluation writes its
+  // unit's K/V into its own session's scratch rows
+  for (int i = 0; i < 2 * n_pairs; ++i) {
+    if ((rc = session_ok(h, ids[i]))) return rc;
+    for (int j = 0; j < i; ++j)
+      if (ids[j] == ids[i]) return SFM_EINVAL;
+  }
+  if ((rc = check_taus(taus, n_taus))) return rc;
+  Guidance gd;
+  gd.on = true;
+  gd.scale = scale;
+  return solve(h, 2 * n_pairs, ids, zs, taus, n_taus, vs, (cudaStream_t)stream, gd);
+}
+
+int sfm_fm_solve_guided(sfm_handle* h, int session, int uncond_session, float* z,
+                        const float* taus, int n_taus, float scale, void* stream) {
+  return sfm_fm_solve_guided_batched(h, 1, &session, &uncond_session, &z, taus, n_taus, scale,
+                                     nullptr, stream);
 }
 
 // The standalone call chooses its split count for a 148-SM B200 whatever the

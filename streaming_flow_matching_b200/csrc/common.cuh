@@ -82,7 +82,8 @@ int launch_rope_scatter(const BatchDesc& b, const float* qkv, const float* cos_t
                         int n_heads, int head_dim, int dtype, cudaStream_t s);
 int launch_head_euler(const BatchDesc& b, const float* x, const void* g, const void* w_out,
                       float* const* z, float* const* v_out, float dtau, int d, int c_lat,
-                      float eps, int dtype, cudaStream_t s);
+                      float eps, int dtype, cudaStream_t s, bool guided = false,
+                      float scale = 1.f);
 int launch_euler(float* z, const float* v, float dtau, long long n, cudaStream_t s);
 
 // GEMM C = A B^T, A [M][K], B [N][K] (both K-contiguous).

@@ -344,6 +344,11 @@ int launch_rope_scatter(const BatchDesc& b, const float* qkv, const float* cos_t
 // halving exchanges (each step hands half of the values to the partner lane),
 // which leaves 2 totals per lane after 62 shuffles; warps then combine
 // through shared memory.
+//
+// Guided (classifier-free guidance, "Wan-Streamer" v0.1 blog, training Stage 3):
+// batch entries 2p and 2p + 1 are the conditional and unconditional evaluations
+// at the same z.  A CTA then takes tokens j, j + 1 of both entries (its 4 rows),
+// forms v = v_u + s (v_c - v_u) per token and updates entry 2p's z once.
 // ---------------------------------------------------------------------------
 constexpr int kHeadRows = 4, kHeadThreads = 256, kHeadCh = 16;
 constexpr int kHeadVals = kHeadRows * kHeadCh;   // 64 accumulators per thread
@@ -370,18 +375,40 @@ __device__ __forceinline__ void halve_step(float* acc, int lane, int o) {
   }
 }
 
-template <typename T>
+template <typename T, bool GUIDED>
 __global__ void __launch_bounds__(kHeadThreads)
     head_euler_kernel(const __grid_constant__ BatchDesc b, const float* __restrict__ x, const T* __restrict__ g,
                       const T* __restrict__ w_out, const __grid_constant__ PtrTable z,
                       const __grid_constant__ PtrTable v_out, float dtau, int d,
-                      int c_lat, float eps) {
+                      int c_lat, float eps, float scale) {
   __shared__ float red[kHeadThreads / 32][kHeadVals];
   __shared__ float red_ss[kHeadThreads / 32][kHeadRows];
-  const int rows = b.n * b.n_tok;
-  const int row0 = blockIdx.x * kHeadRows;
+  __shared__ float vsh[GUIDED ? kHeadVals : 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nr = rows - row0 < kHeadRows ? rows - row0 : kHeadRows;
+  // the CTA's rows of x: consecutive rows, or (guided) tokens j0, j0 + 1 of the
+  // conditional entry 2p followed by the same tokens of the unconditional entry
+  long long xrow[kHeadRows];
+  bool live[kHeadRows];
+  int pair = 0, j0 = 0;
+  if (GUIDED) {
+    const int per_pair = (b.n_tok + 1) / 2;
+    pair = blockIdx.x / per_pair;
+    j0 = (blockIdx.x - pair * per_pair) * 2;
+#pragma unroll
+    for (int q = 0; q < kHeadRows; ++q) {
+      const int j = j0 + (q & 1);
+      live[q] = j < b.n_tok;
+      xrow[q] = (long long)(2 * pair + (q >> 1)) * b.n_tok + (live[q] ? j : 0);
+    }
+  } else {
+    const int rows = b.n * b.n_tok;
+    const int row0 = blockIdx.x * kHeadRows;
+#pragma unroll
+    for (int q = 0; q < kHeadRows; ++q) {
+      live[q] = row0 + q < rows;
+      xrow[q] = live[q] ? row0 + q : row0;
+    }
+  }
   for (int c0 = 0; c0 < c_lat; c0 += kHeadCh) {
     const int nc = c_lat - c0 < kHeadCh ? c_lat - c0 : kHeadCh;
     float acc[kHeadVals];
@@ -395,8 +422,8 @@ __global__ void __launch_bounds__(kHeadThreads)
       load4(g + i, gi);
 #pragma unroll
       for (int q = 0; q < kHeadRows; ++q) {
-        if (q < nr) {
-          load4(x + (size_t)(row0 + q) * d + i, xv[q]);
+        if (live[q]) {
+          load4(x + (size_t)xrow[q] * d + i, xv[q]);
         } else {
           xv[q][0] = xv[q][1] = xv[q][2] = xv[q][3] = 0.f;
         }
@@ -443,11 +470,26 @@ __global__ void __launch_bounds__(kHeadThreads)
         dot += red[w][threadIdx.x];
         sq += red_ss[w][q];
       }
-      const int row = row0 + q;
-      if (q < nr && c < nc) {
-        const float v = dot * rsqrtf(sq / (float)d + eps);
+      const float v = dot * rsqrtf(sq / (float)d + eps);
+      if (GUIDED) {
+        vsh[threadIdx.x] = v;
+      } else if (blockIdx.x * kHeadRows + q < b.n * b.n_tok && c < nc) {
+        const int row = blockIdx.x * kHeadRows + q;
         const int sess = row / b.n_tok;
         const int j = row - sess * b.n_tok;
+        float* zr = z.p[sess] + (size_t)j * c_lat + c0 + c;
+        *zr = fmaf(dtau, v, *zr);
+        if (v_out.p[sess]) v_out.p[sess][(size_t)j * c_lat + c0 + c] = v;
+      }
+    }
+    if (GUIDED) {
+      __syncthreads();
+      // threads 0..31: token j0 + (t / 16), channel c0 + (t % 16)
+      const int t = threadIdx.x, q = t / kHeadCh, c = t % kHeadCh;
+      if (t < 2 * kHeadCh && j0 + q < b.n_tok && c < nc) {
+        const float vc = vsh[q * kHeadCh + c], vu = vsh[(q + 2) * kHeadCh + c];
+        const float v = fmaf(scale, vc - vu, vu);
+        const int sess = 2 * pair, j = j0 + q;
         float* zr = z.p[sess] + (size_t)j * c_lat + c0 + c;
         *zr = fmaf(dtau, v, *zr);
         if (v_out.p[sess]) v_out.p[sess][(size_t)j * c_lat + c0 + c] = v;
@@ -459,23 +501,27 @@ __global__ void __launch_bounds__(kHeadThreads)
 
 int launch_head_euler(const BatchDesc& b, const float* x, const void* g, const void* w_out,
                       float* const* z, float* const* v_out, float dtau, int d, int c_lat,
-                      float eps, int dtype, cudaStream_t s) {
+                      float eps, int dtype, cudaStream_t s, bool guided, float scale) {
   PtrTable zt{}, vt{};
   for (int i = 0; i < b.n; ++i) {
     zt.p[i] = z[i];
     vt.p[i] = v_out ? v_out[i] : nullptr;
   }
+  if (guided && (b.n % 2 || b.n_tok < 1)) return SFM_EINVAL;
   const int rows = b.n * b.n_tok;
-  const int blocks = (rows + kHeadRows - 1) / kHeadRows;
+  const int blocks = guided ? (b.n / 2) * ((b.n_tok + 1) / 2) : (rows + kHeadRows - 1) / kHeadRows;
   if (blocks == 0) return SFM_OK;
   if (d % 4 || ((uintptr_t)g & 15u) || ((uintptr_t)w_out & 15u) || ((uintptr_t)x & 15u))
     return SFM_EUNSUPPORTED;
-  if (dtype == SFM_DTYPE_BF16)
-    head_euler_kernel<__nv_bfloat16><<<blocks, kHeadThreads, 0, s>>>(
-        b, x, (const __nv_bfloat16*)g, (const __nv_bfloat16*)w_out, zt, vt, dtau, d, c_lat, eps);
-  else
-    head_euler_kernel<float><<<blocks, kHeadThreads, 0, s>>>(b, x, (const float*)g, (const float*)w_out,
-                                                    zt, vt, dtau, d, c_lat, eps);
+  if (dtype == SFM_DTYPE_BF16) {
+    auto k = guided ? head_euler_kernel<__nv_bfloat16, true> : head_euler_kernel<__nv_bfloat16, false>;
+    k<<<blocks, kHeadThreads, 0, s>>>(b, x, (const __nv_bfloat16*)g, (const __nv_bfloat16*)w_out, zt,
+                                      vt, dtau, d, c_lat, eps, scale);
+  } else {
+    auto k = guided ? head_euler_kernel<float, true> : head_euler_kernel<float, false>;
+    k<<<blocks, kHeadThreads, 0, s>>>(b, x, (const float*)g, (const float*)w_out, zt, vt, dtau, d,
+                                      c_lat, eps, scale);
+  }
   return record_cuda(cudaGetLastError());
 }
 

@@ -5,6 +5,7 @@
   python -m streaming_flow_matching_b200.microbench euler [--n 268435456]
   python -m streaming_flow_matching_b200.microbench linear --m 924 --n 12288 --k 3072 [--epilogue gelu]
   python -m streaming_flow_matching_b200.microbench step [--layers 1 --cache-units 4]
+  python -m streaming_flow_matching_b200.microbench guided --cache-units 48 [--steps 4 --scale 5]
   python -m streaming_flow_matching_b200.microbench sweep      # attention + append sweep
 
 Inputs are seeded and larger than L2 where the case allows; each timing is
@@ -130,9 +131,45 @@ def bench_step(layers, cache_units, warmup, reps):
             "ms": ms}
 
 
+def bench_guided(layers, cache_units, n_steps, scale, warmup, reps):
+    """Classifier-free-guided solve at the 640x368 unit (conditional session with a full
+    cache_units-unit cache, unconditional session with an empty cache) next to the plain
+    solve of the same session: both timed as whole solves of n_steps Euler steps."""
+    w = S.V02.replace(name=f"v0.2-{layers}L", n_layers=layers, cache_units=cache_units)
+    dev = torch.device("cuda", 0)
+    weights = S.make_weights(w, device=dev)
+    pool = cache_units * w.unit_kv_tokens + w.n_tokens + w.unit_kv_tokens + w.n_tokens
+    p = Performer.from_workload(w, weights, pool_tokens=pool, max_sessions=2)
+    s_id = p.open_session(cache_units)
+    u_id = p.open_session(1)
+    k, v = S.make_kv_slices(w, cache_units, device=dev)
+    p.kvcache_append(s_id, k, v)
+    del k, v
+    _, eps = S.make_latents(w, device=dev)
+    taus = S.uniform_taus(n_steps)
+    z = eps[0].clone()
+
+    def plain():
+        z.copy_(eps[0])
+        p.fm_solve(s_id, z, taus)
+
+    def guided():
+        z.copy_(eps[0])
+        p.fm_solve_guided(s_id, u_id, z, taus, scale)
+
+    ms_plain = _time(plain, warmup, reps)
+    ms_guided = _time(guided, warmup, reps)
+    p.check_device_error()
+    return {"case": "guided", "layers": layers, "cache_tokens": cache_units * w.unit_kv_tokens,
+            "steps": n_steps, "scale": scale, "ms_guided_solve": ms_guided,
+            "ms_plain_solve": ms_plain, "guided_over_plain": ms_guided / ms_plain,
+            "guided_steps_per_s": n_steps / ms_guided * 1e3}
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attention", "append", "euler", "linear", "step", "sweep"])
+    ap.add_argument("case", choices=["attention", "append", "euler", "linear", "step", "guided",
+                                    "sweep"])
     ap.add_argument("--cache-units", type=int, default=4)
     ap.add_argument("--m", type=int, default=924)
     ap.add_argument("--k", type=int, default=3072)
@@ -143,6 +180,8 @@ def main():
     ap.add_argument("--layers", type=int, default=28)
     ap.add_argument("--units", type=int, default=1)
     ap.add_argument("--n", type=int, default=1 << 28)
+    ap.add_argument("--steps", type=int, default=4)
+    ap.add_argument("--scale", type=float, default=5.0)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--reps", type=int, default=10)
     a = ap.parse_args()
@@ -158,6 +197,8 @@ def main():
         out.append(bench_linear(a.m, a.n, a.k, a.epilogue, a.warmup, a.reps))
     elif a.case == "step":
         out.append(bench_step(a.layers, a.cache_units, a.warmup, a.reps))
+    elif a.case == "guided":
+        out.append(bench_guided(a.layers, a.cache_units, a.steps, a.scale, a.warmup, a.reps))
     else:
         for m, n, k, e in [(924, 9216, 3072, "f32"), (924, 3072, 3072, "resid"),
                            (924, 12288, 3072, "gelu"), (924, 3072, 12288, "resid")]:

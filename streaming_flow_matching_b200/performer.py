@@ -136,6 +136,36 @@ class Performer:
         L.check(L.lib.sfm_fm_solve_batched(self._h, n, s, zp, t, len(taus), _stream()),
                 "sfm_fm_solve_batched")
 
+    def fm_solve_guided(self, session, uncond_session, z, taus, scale):
+        """Classifier-free-guided solve: v = v_u + scale (v_c - v_u) at every step."""
+        _need(z, torch.float32, "z", (self.n_tok, self.shape["c_lat"]))
+        t = (C.c_float * len(taus))(*taus)
+        L.check(L.lib.sfm_fm_solve_guided(self._h, session, uncond_session, _ptr(z), t, len(taus),
+                                          scale, _stream()), "sfm_fm_solve_guided")
+
+    def fm_solve_guided_batched(self, sessions, uncond_sessions, zs, taus, scale, v_outs=None):
+        """Guided solves of len(sessions) pairs in one batch; v_outs (optional) receive
+        the last step's guided velocities."""
+        n = len(sessions)
+        if len(uncond_sessions) != n or len(zs) != n:
+            raise ValueError("sessions, uncond_sessions and zs differ in length")
+        for z in zs:
+            _need(z, torch.float32, "z", (self.n_tok, self.shape["c_lat"]))
+        vp = None
+        if v_outs is not None:
+            if len(v_outs) != n:
+                raise ValueError("v_outs and sessions differ in length")
+            for v in v_outs:
+                if v is not None:
+                    _need(v, torch.float32, "v_out", (self.n_tok, self.shape["c_lat"]))
+            vp = (C.c_void_p * n)(*[_ptr(v) for v in v_outs])
+        s = (C.c_int * n)(*sessions)
+        u = (C.c_int * n)(*uncond_sessions)
+        zp = (C.c_void_p * n)(*[z.data_ptr() for z in zs])
+        t = (C.c_float * len(taus))(*taus)
+        L.check(L.lib.sfm_fm_solve_guided_batched(self._h, n, s, u, zp, t, len(taus), scale, vp,
+                                                  _stream()), "sfm_fm_solve_guided_batched")
+
     def set_graph_mode(self, enabled):
         """Solves as one captured CUDA graph (True, the default) or direct launches."""
         L.check(L.lib.sfm_set_graph_mode(self._h, 1 if enabled else 0), "sfm_set_graph_mode")

@@ -79,3 +79,39 @@ def test_graph_batched_solve_matches_direct_launches(cuda_device):
         assert torch.equal(a, b)
     p.check_device_error()
     p.close()
+
+
+def test_graph_guided_solves_alternating_with_plain_ones_match_direct(cuda_device):
+    # plain and guided solves keep separate executable graphs; alternating them
+    # must give what direct launches give
+    from streaming_flow_matching_b200 import Performer
+    w = SMALL_BF16
+    weights = to_cuda(S.make_weights(w))
+    caps = [3, 1]
+    pool = sum(c * w.unit_kv_tokens + w.n_tokens for c in caps)
+    p = Performer.from_workload(w, weights, pool_tokens=pool, max_sessions=2)
+    s = p.open_session(3)
+    u = p.open_session(1)
+    k, v = S.make_kv_slices(w, 3)
+    p.kvcache_append(s, k.cuda(), v.cuda())
+    _, eps = S.make_latents(w)
+    eps = eps[0].cuda()
+    taus = S.uniform_taus(w.n_steps)
+    res = []
+    for graph in (False, True):
+        p.set_graph_mode(graph)
+        out = []
+        for scale in (3.0, None, 1.5, None):
+            z = eps.clone()
+            if scale is None:
+                p.fm_solve(s, z, taus)
+            else:
+                p.fm_solve_guided(s, u, z, taus, scale)
+            torch.cuda.synchronize()
+            out.append(z.cpu())
+        res.append(out)
+    for i, (a, b) in enumerate(zip(*res)):
+        assert torch.equal(a, b), f"call {i}"
+    assert not torch.equal(res[1][0], res[1][2])     # the scale reaches the graph
+    p.check_device_error()
+    p.close()

@@ -250,6 +250,25 @@ SFM_API int sfm_attention(const void* q, const void* k, const void* v, void* o, 
                   size_t workspace_bytes, void* stream);
 
 /*
+ * General block-causal attention ("Wan-Streamer" v0.1 blog, §3.3: a unit sees
+ * itself bidirectionally and every earlier unit, never a later one), the form
+ * a multi-unit pass such as a scene prefill needs.  The n_q queries are
+ * n_q / unit_tokens units of unit_tokens tokens (the last one may be shorter);
+ * the last n_q of the n_kv keys are theirs, in the same order, and the first
+ * n_kv - n_q keys are a prefix (earlier context, e.g. a cache) every query
+ * sees.  Query i attends to keys [0, n_kv - n_q + min((i / unit_tokens + 1) *
+ * unit_tokens, n_q)).  unit_tokens >= n_q gives sfm_attention's result (every
+ * key visible).  Layouts, dtypes, workspace (same size as for sfm_attention)
+ * and errors as for sfm_attention; SFM_EINVAL if unit_tokens < 1 or
+ * n_kv < n_q.  Key tiles past a query block's last visible key are skipped,
+ * so the causal half of the work is not done.
+ */
+SFM_API int sfm_attention_block_causal(const void* q, const void* k, const void* v, void* o,
+                                       int n_q, int n_kv, int unit_tokens, int n_heads,
+                                       int head_dim, int dtype, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/*
  * sfm_attention without any allocation.  No counterpart in the paper: this
  * entry point exists for callers that cannot allocate device memory where they
  * need attention -- a real-time serving loop with a hard per-unit deadline

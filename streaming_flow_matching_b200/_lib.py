@@ -73,6 +73,7 @@ def _load():
         "sfm_set_graph_mode": (i, [vp, i]),
         "sfm_attention_workspace_bytes": (sz, [i, i, i, i, i]),
         "sfm_attention": (i, [vp, vp, vp, vp, i, i, i, i, i, vp, sz, vp]),
+        "sfm_attention_block_causal": (i, [vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]),
         "sfm_attention_noalloc": (i, [vp, vp, vp, vp, i, i, i, i, i, vp]),
         "sfm_linear": (i, [vp, vp, vp, i, i, i, i, i, vp]),
         "sfm_check_device_error": (i, [vp, C.POINTER(i)]),
@@ -98,7 +99,7 @@ EXPORTS = ["sfm_create", "sfm_destroy", "sfm_session_open", "sfm_session_reset",
            "sfm_session_get_info", "sfm_kvcache_append", "sfm_kvcache_read", "sfm_denoise_step",
            "sfm_fm_solve", "sfm_fm_solve_batched", "sfm_fm_solve_guided",
            "sfm_fm_solve_guided_batched", "sfm_set_graph_mode", "sfm_attention_workspace_bytes",
-           "sfm_attention", "sfm_attention_noalloc", "sfm_linear", "sfm_euler_update", "sfm_profile_begin", "sfm_profile_end",
+           "sfm_attention", "sfm_attention_block_causal", "sfm_attention_noalloc", "sfm_linear", "sfm_euler_update", "sfm_profile_begin", "sfm_profile_end",
            "sfm_kernel_launch_count", "sfm_check_device_error", "sfm_strerror",
            "sfm_last_cuda_error"]
 

@@ -741,9 +741,15 @@ size_t sfm_attention_workspace_bytes(int n_q, int n_kv, int n_heads, int head_di
   return attention_workspace_bytes(n_q, n_heads, splits);
 }
 
-int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q, int n_kv,
-                  int n_heads, int head_dim, int dtype, void* workspace, size_t workspace_bytes,
-                  void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Standalone attention, every key visible (unit_tokens = 0) or block-causal over
+// query units of unit_tokens with the first n_kv - n_q keys a shared prefix.
+int attention_call(const void* q, const void* k, const void* v, void* o, int n_q, int n_kv,
+                   int unit_tokens, int n_heads, int head_dim, int dtype, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k || !v || !o || n_q < 1 || n_kv < 1 || n_heads < 1) return SFM_EINVAL;
   if (dtype != SFM_DTYPE_BF16 && dtype != SFM_DTYPE_FP32) return SFM_EINVAL;
   if (dtype == SFM_DTYPE_BF16 && head_dim != 128) return SFM_EUNSUPPORTED;
@@ -755,11 +761,11 @@ int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q,
   AttnDesc a{};
   a.n = 1;
   a.rows_per = n_q;
+  a.unit_rows = unit_tokens;
   a.kbase[0] = 0;
   a.nkeys[0] = n_kv;
   if (dtype == SFM_DTYPE_FP32)
-    return launch_attention(a, q, k, v, o, n_heads, head_dim, dtype, 1, nullptr, nullptr,
-                            (cudaStream_t)stream);
+    return launch_attention(a, q, k, v, o, n_heads, head_dim, dtype, 1, nullptr, nullptr, stream);
   const int splits = attention_tc_splits(n_q, 1, n_kv, n_heads, kStandaloneSms);
   float *o_part = nullptr, *lse_part = nullptr;
   if (splits > 1) {
@@ -772,7 +778,26 @@ int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q,
   if (!rc) rc = make_rows_map(&mv, v, n_kv, n_heads, kAttnKVBoxRows);
   if (rc) return rc;
   return launch_attention_tc(mq, mk, mv, a, 0, n_heads, splits, o, o_part, lse_part, nullptr,
-                             (cudaStream_t)stream);
+                             stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int sfm_attention(const void* q, const void* k, const void* v, void* o, int n_q, int n_kv,
+                  int n_heads, int head_dim, int dtype, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  return attention_call(q, k, v, o, n_q, n_kv, 0, n_heads, head_dim, dtype, workspace,
+                        workspace_bytes, (cudaStream_t)stream);
+}
+
+int sfm_attention_block_causal(const void* q, const void* k, const void* v, void* o, int n_q,
+                               int n_kv, int unit_tokens, int n_heads, int head_dim, int dtype,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (unit_tokens < 1 || n_kv < n_q) return SFM_EINVAL;
+  return attention_call(q, k, v, o, n_q, n_kv, unit_tokens, n_heads, head_dim, dtype, workspace,
+                        workspace_bytes, (cudaStream_t)stream);
 }
 
 int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream) {

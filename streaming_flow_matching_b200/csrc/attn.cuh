@@ -14,12 +14,25 @@ constexpr int kAttnKVBoxRows = 128;
 
 // Query rows [s * rows_per, (s + 1) * rows_per) of session s attend to key
 // rows [kbase[s], kbase[s] + nkeys[s]) of the layer's K/V arrays.
+// unit_rows = 0: every key is visible to every query (the performer form).
+// unit_rows = U > 0: block-causal over units of U queries -- the last rows_per
+// keys belong to the queries themselves, the keys before them are a prefix
+// every query sees, and query i (of its session) sees the prefix plus the keys
+// of units <= i / U:  keys [0, attn_key_limit(...)).
 struct AttnDesc {
   int n;
   int rows_per;
+  int unit_rows;
   long long kbase[kMaxBatch];
   int nkeys[kMaxBatch];
 };
+
+__host__ __device__ __forceinline__ int attn_key_limit(int nkeys, int rows_per, int unit_rows,
+                                                       int i) {
+  if (unit_rows <= 0) return nkeys;
+  const int own = (i / unit_rows + 1) * unit_rows;
+  return nkeys - rows_per + (own < rows_per ? own : rows_per);
+}
 
 size_t attention_workspace_bytes(long long rows, int n_heads, int n_splits);
 int launch_attention(const AttnDesc& a, const void* q, const void* k, const void* v, void* o,

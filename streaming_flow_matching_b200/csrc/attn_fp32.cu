@@ -1,7 +1,9 @@
 // Attention of the current unit over [valid cache ; current unit] -- the
 // performer form of the block-causal attention of "Wan-Streamer" v0.1 blog
 // §3.3: every cached unit precedes the current one and the current unit is
-// bidirectional, so every key is visible to every query.
+// bidirectional, so every key is visible to every query.  With
+// AttnDesc::unit_rows > 0 the general block-causal form: several units of
+// queries, each seeing the shared prefix and the units up to its own.
 //
 //   fp32 mode: one warp per (query row, head) on the CUDA cores.
 //   attn_merge_kernel: combines the split-KV partial results of the tcgen05
@@ -30,7 +32,9 @@ __global__ void attn_f32_kernel(AttnDesc a, const float* __restrict__ q,
   for (int e = 0; e < ne; ++e) qv[e] = q[row * ld + h * D + lane + 32 * e];
   float m = -INFINITY, l = 0.f;
   const long long kb = a.kbase[sess];
-  for (int t = 0; t < a.nkeys[sess]; ++t) {
+  const int lim = attn_key_limit(a.nkeys[sess], a.rows_per, a.unit_rows,
+                                 (int)(row - (long long)sess * a.rows_per));
+  for (int t = 0; t < lim; ++t) {
     const float* kr = k + (kb + t) * ld + h * D;
     float s = 0.f;
     for (int e = 0; e < ne; ++e) s = fmaf(qv[e], kr[lane + 32 * e], s);

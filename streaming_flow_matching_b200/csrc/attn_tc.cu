@@ -27,6 +27,13 @@
 // The last, partial key tile is masked in S, and its V rows past the key range
 // are zeroed in shared memory before P V, so rows outside the range never
 // contribute (whatever they hold).
+// Block-causal form (AttnDesc::unit_rows > 0, several query units over a shared
+// prefix): a CTA walks the key tiles up to its last row's limit, and each
+// softmax thread masks the logits past its own row's limit, so keys of later
+// units are neither loaded by CTAs that cannot see them nor seen by rows that
+// may not.  A row can then have no visible key in a whole split: its running
+// max stays -inf, its partial is 0 with log-sum-exp -inf, and the merge gives
+// it weight 0.
 #include <math.h>
 
 #include "attn.cuh"
@@ -94,7 +101,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int qb = blockIdx.x - sess * args.qtiles;
   const int h = blockIdx.y, split = blockIdx.z;
   const long long row0 = (long long)sess * args.a.rows_per + (long long)qb * ROWS;
-  const int nkeys = args.a.nkeys[sess];
+  // keys of this CTA: up to the limit of its last query row (block-causal: the
+  // rows' own limits are masked per row below)
+  const int q_last = min(args.a.rows_per, qb * ROWS + ROWS) - 1;
+  const int nkeys = attn_key_limit(args.a.nkeys[sess], args.a.rows_per, args.a.unit_rows, q_last);
   const long long kbase = args.a.kbase[sess];
   const int ntiles = (nkeys + BKV - 1) / BKV;
   const int tps = (ntiles + args.n_splits - 1) / args.n_splits;
@@ -266,6 +276,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t col_s = (uint32_t)(t * 256), col_o = col_s + 128;
     const int q_rows = min(BQ, args.a.rows_per - qb * ROWS - t * BQ);   // may be <= 0
+    // this row's key limit (rows past the session's end take the last row's)
+    const int my_keys = attn_key_limit(args.a.nkeys[sess], args.a.rows_per, args.a.unit_rows,
+                                       min(qb * ROWS + t * BQ + r, args.a.rows_per - 1));
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     const float sc = args.scale_log2;
@@ -276,17 +289,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_after();
       const int kvalid = nkeys - (t0 + j) * BKV;         // > 0; < BKV only on the last tile
-      if (kvalid < BKV) {
-        // partial tile (CTA-uniform): overwrite the logits past the key range with -inf
+      const int kmine = my_keys - (t0 + j) * BKV;        // this row's; may be <= 0
+      const int kwarp = __reduce_min_sync(0xffffffffu, kmine);
+      if (kwarp < BKV) {
+        // partial tile for some row of the warp: overwrite the row's logits past its
+        // key limit with -inf (the TMEM accesses are warp-collective)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          if (c * 32 + 32 <= kvalid) continue;
+          if (c * 32 + 32 <= kwarp) continue;
           uint32_t u[32];
           tmem_ld32(tmem + lane_base + col_s + c * 32, u);
           tmem_wait_ld(u);
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (c * 32 + i >= kvalid) u[i] = __float_as_uint(-INFINITY);
+            if (c * 32 + i >= kmine) u[i] = __float_as_uint(-INFINITY);
           tmem_st32(tmem + lane_base + col_s + c * 32, u);
         }
         tmem_st_wait();
@@ -302,7 +318,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       float mx = -INFINITY;
       bool fresh = j == 0;                                // P still to be computed
       if (!fresh) {
-        const float neg_m = -m;
+        // a row with no visible key so far (block-causal, a later split) has m = -inf:
+        // its attempt below is dropped by the rescale test, so any finite base serves
+        const float neg_m = m == -INFINITY ? 0.f : -m;
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         uint32_t u[2][32];
         tmem_ld32(tmem + lane_base + col_s, u[0]);
@@ -326,7 +344,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
           // O_t's previous P V has completed (S_t(j) was issued after it): rescale it
           const float m_new = fmaxf(m, mx);
-          const float alpha = ex2_approx(m - m_new);
+          const float alpha = m == -INFINITY ? 0.f : ex2_approx(m - m_new);   // O, l are 0 then
           l *= alpha;
           m = m_new;
 #pragma unroll
@@ -362,7 +380,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
       }
       if (__any_sync(0xffffffffu, fresh)) {
-        const float neg_m = -m;
+        const float neg_m = m == -INFINITY ? 0.f : -m;   // every key of the row masked: p = 0
         l4[0] = l4[1] = l4[2] = l4[3] = 0.f;
         uint32_t u[2][32];
         tmem_ld32(tmem + lane_base + col_s, u[0]);

@@ -1,6 +1,7 @@
 """Micro-benchmarks of single kernels of the hot path, timed with CUDA events.
 
   python -m streaming_flow_matching_b200.microbench attention --n-kv 16800 [--n-q 924 --heads 24]
+  python -m streaming_flow_matching_b200.microbench attention --n-q 3696 --n-kv 61296 --unit-tokens 924
   python -m streaming_flow_matching_b200.microbench append [--layers 28 --units 1]
   python -m streaming_flow_matching_b200.microbench euler [--n 268435456]
   python -m streaming_flow_matching_b200.microbench linear --m 924 --n 12288 --k 3072 [--epilogue gelu]
@@ -41,6 +42,8 @@ def _peaks():
 
 
 def _time(fn, warmup, reps):
+    """Median of `reps` single calls, each bracketed by events (host work of the call
+    included when the GPU waits for it)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -55,17 +58,46 @@ def _time(fn, warmup, reps):
     return statistics.median(ts)
 
 
-def bench_attention(n_q, n_kv, heads, warmup, reps):
+def _time_b2b(fn, reps):
+    """Mean device time per call over `reps` calls enqueued back to back (the host runs
+    ahead of the GPU, so gaps between launches vanish unless a call's host work is
+    longer than its kernels)."""
+    fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def bench_attention(n_q, n_kv, heads, warmup, reps, unit=None):
+    """unit: None for every key visible; else block-causal over query units of `unit`
+    tokens (the first n_kv - n_q keys a shared prefix).  FLOPs count the visible
+    keys only: 4 D H per (query, visible key)."""
     q, k, v = S.make_qkv(n_q, n_kv, heads, 128, device="cuda")
     o = torch.empty_like(q)
     ws_n = attention_workspace_bytes(n_q, n_kv, heads, 128)
     ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda")
-    ms = _time(lambda: attention(q, k, v, o, ws), warmup, reps)
-    flop = 4.0 * n_q * n_kv * heads * 128
+    call = lambda: attention(q, k, v, o, ws, unit_tokens=unit)  # noqa: E731
+    ms_single = _time(call, warmup, reps)
+    ms = _time_b2b(call, max(reps, 20))
+    if unit is None:
+        visible = n_q * n_kv
+    else:
+        prefix = n_kv - n_q
+        visible = sum(prefix + min((i // unit + 1) * unit, n_q) for i in range(n_q))
+    flop = 4.0 * visible * heads * 128
     hbm, bf16, src = _peaks()
     tf = flop / (ms / 1e3) / 1e12
-    return {"case": "attention", "n_q": n_q, "n_kv": n_kv, "heads": heads, "ms": ms,
-            "tflops": tf, "frac_of_bf16_burst": tf / bf16, "peak_source": src}
+    out = {"case": "attention", "n_q": n_q, "n_kv": n_kv, "heads": heads, "ms": ms,
+           "ms_single_call": ms_single, "tflops": tf, "frac_of_bf16_burst": tf / bf16,
+           "peak_source": src, "timing": "ms: back-to-back mean; ms_single_call: median"}
+    if unit is not None:
+        out.update({"unit_tokens": unit, "visible_fraction": visible / (n_q * n_kv)})
+    return out
 
 
 def bench_append(layers, units, warmup, reps):
@@ -177,6 +209,8 @@ def main():
     ap.add_argument("--n-q", type=int, default=924)
     ap.add_argument("--n-kv", type=int, default=57600 + 924)
     ap.add_argument("--heads", type=int, default=24)
+    ap.add_argument("--unit-tokens", type=int, default=None,
+                    help="attention: block-causal over query units of this many tokens")
     ap.add_argument("--layers", type=int, default=28)
     ap.add_argument("--units", type=int, default=1)
     ap.add_argument("--n", type=int, default=1 << 28)
@@ -188,7 +222,7 @@ def main():
     torch.cuda.set_device(0)
     out = []
     if a.case == "attention":
-        out.append(bench_attention(a.n_q, a.n_kv, a.heads, a.warmup, a.reps))
+        out.append(bench_attention(a.n_q, a.n_kv, a.heads, a.warmup, a.reps, a.unit_tokens))
     elif a.case == "append":
         out.append(bench_append(a.layers, a.units, a.warmup, a.reps))
     elif a.case == "euler":

@@ -188,8 +188,14 @@ class Performer:
             pass
 
 
-def attention(q, k, v, out=None, workspace=None):
-    """O = softmax(Q K^T / sqrt(D)) V per head, every key visible; q [n_q][H][D], k/v [n_kv][H][D]."""
+def attention(q, k, v, out=None, workspace=None, unit_tokens=None):
+    """O = softmax(Q K^T / sqrt(D)) V per head; q [n_q][H][D], k/v [n_kv][H][D].
+
+    unit_tokens None: every key visible.  Otherwise block-causal: the queries are
+    units of unit_tokens tokens whose own keys are the last n_q keys, the first
+    n_kv - n_q keys are a prefix all of them see, and a query sees the keys of
+    its own and earlier units only.
+    """
     dt = _DT[q.dtype]
     _need(q, q.dtype, "q")
     _need(k, q.dtype, "k")
@@ -202,8 +208,13 @@ def attention(q, k, v, out=None, workspace=None):
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    L.check(L.lib.sfm_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), n_q, n_kv, H, D, dt,
-                                _ptr(workspace), ws_bytes, _stream()), "sfm_attention")
+    if unit_tokens is None:
+        L.check(L.lib.sfm_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), n_q, n_kv, H, D, dt,
+                                    _ptr(workspace), ws_bytes, _stream()), "sfm_attention")
+    else:
+        L.check(L.lib.sfm_attention_block_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(out), n_q, n_kv,
+                                                 unit_tokens, H, D, dt, _ptr(workspace), ws_bytes,
+                                                 _stream()), "sfm_attention_block_causal")
     return out
 
 

@@ -68,6 +68,8 @@ def test_null_arguments_are_rejected():
     assert L.lib.sfm_attention(None, None, None, None, 4, 4, 1, 128, 0, None, 0, None) == L.SFM_EINVAL
     assert L.lib.sfm_attention_workspace_bytes(924, 58524, 24, 128, L.SFM_DTYPE_FP32) == 0
     assert L.lib.sfm_set_graph_mode(None, 1) == L.SFM_EINVAL
+    assert L.lib.sfm_attention_block_causal(None, None, None, None, 4, 4, 2, 1, 128, 0, None, 0,
+                                            None) == L.SFM_EINVAL
     taus = (C.c_float * 2)(1.0, 0.0)
     assert L.lib.sfm_fm_solve_guided(None, 0, 1, None, taus, 2, 3.0, None) == L.SFM_EINVAL
     assert L.lib.sfm_fm_solve_guided_batched(None, 1, None, None, None, taus, 2, 3.0, None,

@@ -162,8 +162,8 @@ def test_v02_width_full_cache_step_matches_oracle(cuda_device):
 # attention
 # ---------------------------------------------------------------------------
 
-# up to 256 query rows run on single CTAs, more on CTA pairs (512 rows per pair):
-# 257 leaves the second CTA of the pair without rows, 513 a pair with one row
+# a CTA takes 256 query rows as two 128-row tiles: 257 gives a second CTA with one
+# row (its tile B empty), 300 a partial tile B, 513 a third CTA with one row
 @pytest.mark.parametrize("n_q,n_kv", [(1, 1), (17, 5), (64, 64), (204, 704), (924, 5724),
                                       (257, 1), (300, 129), (513, 1000), (1030, 3000)])
 def test_attention_bf16_matches_oracle(cuda_device, n_q, n_kv):

@@ -766,7 +766,13 @@ int attention_call(const void* q, const void* k, const void* v, void* o, int n_q
   a.nkeys[0] = n_kv;
   if (dtype == SFM_DTYPE_FP32)
     return launch_attention(a, q, k, v, o, n_heads, head_dim, dtype, 1, nullptr, nullptr, stream);
-  const int splits = attention_tc_splits(n_q, 1, n_kv, n_heads, kStandaloneSms);
+  // a block-causal call uses at most the splits of the every-key-visible one, so the
+  // workspace sfm_attention_workspace_bytes sizes serves both
+  int splits = attention_tc_splits(n_q, 1, n_kv, n_heads, kStandaloneSms);
+  if (unit_tokens > 0) {
+    const int bc = attention_tc_splits(n_q, 1, n_kv, n_heads, kStandaloneSms, unit_tokens);
+    splits = bc < splits ? bc : splits;
+  }
   float *o_part = nullptr, *lse_part = nullptr;
   if (splits > 1) {
     o_part = (float*)workspace;

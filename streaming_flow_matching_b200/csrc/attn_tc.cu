@@ -438,27 +438,61 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long ld = (long long)args.H * D;
     const bool have = ok && T > 0 && l > 0.f;
     const float inv = have ? 1.f / l : 0.f;
-    for (int c = 0; c < 4; ++c) {
-      uint32_t u[32];
-      if (T > 0) {
-        tmem_ld32(tmem + lane_base + col_o + c * 32, u);
-        tmem_wait_ld(u);
+    if (ok) {
+      // Stage the warp's 32 normalised rows in shared memory, then write whole rows
+      // (one row per warp instruction: coalesced).  The staging area is the Q and K
+      // stages: the last S MMA of both tiles was issued before this tile's last
+      // P V, whose completion o_done signalled, so nothing reads them any more
+      // (the other tile's last P V may still read a V stage, which stays untouched).
+      // Row `lane` keeps its float4 slot q at q ^ lane: no bank conflicts either way.
+      float4* stage = reinterpret_cast<float4*>(smem + OFF_Q) + (warp - 2) * (32 * 32);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        if (T > 0) {
+          tmem_ld32(tmem + lane_base + col_o + c * 32, u);
+          tmem_wait_ld(u);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) u[i] = 0u;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float4 f;
+          f.x = have ? __uint_as_float(u[4 * q]) * inv : 0.f;
+          f.y = have ? __uint_as_float(u[4 * q + 1]) * inv : 0.f;
+          f.z = have ? __uint_as_float(u[4 * q + 2]) * inv : 0.f;
+          f.w = have ? __uint_as_float(u[4 * q + 3]) * inv : 0.f;
+          stage[lane * 32 + ((c * 8 + q) ^ lane)] = f;
+        }
       }
-      if (r >= q_rows) continue;
-      float o[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] = have ? __uint_as_float(u[i]) * inv : 0.f;
-      if (args.n_splits == 1) {
-        uint4* d = reinterpret_cast<uint4*>(args.o + grow * ld + h * D + c * 32);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          d[q] = make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
-                            pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
-      } else {
-        float4* d = reinterpret_cast<float4*>(args.o_part + ((long long)split * args.total_rows + grow) * ld +
-                                              h * D + c * 32);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) d[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      __syncwarp();
+      const long long grow0 = row0 + t * BQ + quarter * 32;   // global row of the warp's lane 0
+      for (int rr = 0; rr < 32; ++rr) {
+        if (quarter * 32 + rr >= q_rows) break;               // warp-uniform
+        const float4 f = stage[rr * 32 + (lane ^ rr)];        // columns 4 lane .. 4 lane + 3
+        if (args.n_splits == 1) {
+          uint2 b;
+          b.x = pack_bf16x2(f.x, f.y);
+          b.y = pack_bf16x2(f.z, f.w);
+          *reinterpret_cast<uint2*>(args.o + (grow0 + rr) * ld + h * D + 4 * lane) = b;
+        } else {
+          *reinterpret_cast<float4*>(args.o_part + ((long long)split * args.total_rows + grow0 + rr) * ld +
+                                     h * D + 4 * lane) = f;
+        }
+      }
+    } else if (r < q_rows) {
+      // unwinding after a timed-out wait (loads may still land in shared memory):
+      // zeros, written directly
+      for (int c = 0; c < 4; ++c) {
+        if (args.n_splits == 1) {
+          uint4* d = reinterpret_cast<uint4*>(args.o + grow * ld + h * D + c * 32);
+          for (int q = 0; q < 4; ++q) d[q] = make_uint4(0u, 0u, 0u, 0u);
+        } else {
+          float4* d = reinterpret_cast<float4*>(args.o_part + ((long long)split * args.total_rows + grow) * ld +
+                                                h * D + c * 32);
+          for (int q = 0; q < 8; ++q) d[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
     }
     if (r < q_rows && args.n_splits > 1)
@@ -476,20 +510,43 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace atc
 
+// Split count from a cost model of the kernel, in microseconds on a B200:
+//   CTA time  = (key tiles of the CTA) x kStepUs + kCtaUs (set-up, output, hand-over),
+//   kernel    = max(waves x mean CTA time, longest CTA time), waves = ceil(CTAs / SMs),
+//   merge     = its bytes (fp32 partials of every split read, bf16 O written) / kMergeBps.
+// More splits fill the SMs and shorten the longest CTA; each split adds fixed cost and
+// merge traffic.  Block-causal calls count each query block's own key tiles.
 int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads,
-                        int sms) {
-  const long long ctas = (long long)n_sessions * ((rows_per_session + atc::ROWS - 1) / atc::ROWS) * n_heads;
+                        int sms, int unit_rows) {
+  constexpr double kStepUs = 2.0, kCtaUs = 5.0, kMergeBps = 4.0e6;   // bytes per microsecond
+  const int qtiles = (rows_per_session + atc::ROWS - 1) / atc::ROWS;
+  const long long ctas = (long long)n_sessions * qtiles * n_heads;
   const long long tiles = (max_keys + atc::BKV - 1) / atc::BKV;
   int best = 1;
-  double best_eff = 0.0;
+  double best_us = 0.0;
   for (int s = 1; s <= kMaxSplits; ++s) {
     if (s > 1 && tiles / s < 2) break;
+    double sum_t = 0.0, max_t = 0.0;
+    for (int b = 0; b < qtiles; ++b) {
+      const int last = (b + 1) * atc::ROWS < rows_per_session ? (b + 1) * atc::ROWS - 1 : rows_per_session - 1;
+      const long long lim = unit_rows > 0 && max_keys < (1LL << 31)
+                                ? attn_key_limit((int)max_keys, rows_per_session, unit_rows, last)
+                                : max_keys;
+      const double t = (double)(((lim + atc::BKV - 1) / atc::BKV + s - 1) / s) * kStepUs + kCtaUs;
+      sum_t += t;
+      max_t = t > max_t ? t : max_t;
+    }
     const long long work = ctas * s;
-    const long long waves = (work + sms - 1) / sms;
-    const double eff = (double)work / (double)(waves * sms);
-    if (eff > best_eff + 0.04) {
+    const double waves = (double)((work + sms - 1) / sms);
+    double us = waves * sum_t / qtiles;
+    if (max_t > us) us = max_t;
+    if (s > 1) {
+      const double rows = (double)n_sessions * rows_per_session * n_heads;
+      us += (s * rows * (atc::D + 1) * 4.0 + rows * atc::D * 2.0) / kMergeBps;
+    }
+    if (s == 1 || us < best_us) {
       best = s;
-      best_eff = eff;
+      best_us = us;
     }
   }
   return best;

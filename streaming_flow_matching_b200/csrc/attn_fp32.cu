@@ -54,36 +54,35 @@ __global__ void attn_f32_kernel(AttnDesc a, const float* __restrict__ q,
 
 // Merge split-KV partials: one warp per (row, head); D = 128 (float4 per lane).
 // Every split's log-sum-exp and partial row are loaded up front, so the loads
-// of a row are in flight together.
-__global__ void attn_merge_kernel(const float* __restrict__ o_part,
-                                  const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ o,
-                                  long long total_rows, int H, int n_splits) {
+// of a row are in flight together.  The split count is a template parameter so a
+// thread holds exactly its splits' values (a fixed 16-slot version needed 94
+// registers and ran at a quarter of the warps an SM can hold).
+template <int S>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict__ o_part,
+                                                         const float* __restrict__ lse_part,
+                                                         __nv_bfloat16* __restrict__ o,
+                                                         long long total_rows, int H) {
   const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (gw >= total_rows * H) return;
   const long long row = gw / H;
   const int h = (int)(gw - row * H);
   const long long ld = (long long)H * 128;
-  float lse[kMaxSplits];
-  float4 p[kMaxSplits];
+  float lse[S];
+  float4 p[S];
 #pragma unroll
-  for (int s = 0; s < kMaxSplits; ++s) {
-    if (s < n_splits) {
-      lse[s] = __ldcs(lse_part + ((long long)s * total_rows + row) * H + h);
-      p[s] = __ldcs(reinterpret_cast<const float4*>(o_part + ((long long)s * total_rows + row) * ld +
-                                                    h * 128) + lane);
-    } else {
-      lse[s] = -INFINITY;
-      p[s] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+  for (int s = 0; s < S; ++s) {
+    lse[s] = __ldcs(lse_part + ((long long)s * total_rows + row) * H + h);
+    p[s] = __ldcs(reinterpret_cast<const float4*>(o_part + ((long long)s * total_rows + row) * ld +
+                                                  h * 128) + lane);
   }
   float mmax = -INFINITY;
 #pragma unroll
-  for (int s = 0; s < kMaxSplits; ++s) mmax = fmaxf(mmax, lse[s]);
+  for (int s = 0; s < S; ++s) mmax = fmaxf(mmax, lse[s]);
   float wsum = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int s = 0; s < kMaxSplits; ++s) {
+  for (int s = 0; s < S; ++s) {
     // a split without keys has lse = -inf and weight 0 (its partial row is zeros)
     const float w = lse[s] == -INFINITY ? 0.f : exp2f(lse[s] - mmax);
     wsum += w;
@@ -96,6 +95,20 @@ __global__ void attn_merge_kernel(const float* __restrict__ o_part,
   __nv_bfloat16* od = o + row * ld + h * 128 + lane * 4;
   *reinterpret_cast<__nv_bfloat162*>(od) = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
   *reinterpret_cast<__nv_bfloat162*>(od + 2) = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+}
+
+template <int S>
+static void launch_merge_s(const float* o_part, const float* lse_part, void* o, long long total_rows,
+                           int n_heads, int n_splits, cudaStream_t s) {
+  if constexpr (S > 1) {
+    if (n_splits != S) {
+      launch_merge_s<S - 1>(o_part, lse_part, o, total_rows, n_heads, n_splits, s);
+      return;
+    }
+    const long long warps = total_rows * n_heads;
+    attn_merge_kernel<S><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
+        o_part, lse_part, (__nv_bfloat16*)o, total_rows, n_heads);
+  }
 }
 
 size_t attention_workspace_bytes(long long rows, int n_heads, int n_splits) {
@@ -125,9 +138,8 @@ int launch_attention(const AttnDesc& a, const void* q, const void* k, const void
 
 int launch_attention_merge(const float* o_part, const float* lse_part, void* o,
                            long long total_rows, int n_heads, int n_splits, cudaStream_t s) {
-  const long long warps = total_rows * n_heads;
-  attn_merge_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
-      o_part, lse_part, (__nv_bfloat16*)o, total_rows, n_heads, n_splits);
+  if (n_splits < 2 || n_splits > kMaxSplits) return SFM_EINVAL;
+  launch_merge_s<kMaxSplits>(o_part, lse_part, o, total_rows, n_heads, n_splits, s);
   return record_cuda(cudaGetLastError());
 }
 

@@ -310,6 +310,21 @@ SFM_API int sfm_linear(const void* x, const void* w, void* y, int M, int N, int 
 /* Vectorised Euler update z[i] += dtau * v[i], i < n; device fp32. */
 SFM_API int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream);
 
+/*
+ * Test-only closed-form check of the solve loop: the Euler solve of
+ * sfm_fm_solve with f_theta replaced by the exact velocity of the rectified-
+ * flow path ("Wan-Streamer" v0.1 blog, §3.4: z_tau = (1 - tau) z0 + tau eps,
+ * constant velocity eps - z0), written as the state-dependent (z - z0) / tau
+ * and evaluated at each step's starting tau.  From z = eps at taus[0] = 1 any
+ * schedule ends at z0 (up to fp32 rounding); a step that evaluated the velocity
+ * at its end point, or moved the wrong way, would not.  z0, z: device fp32
+ * [N][C] (N, C of the handle's configuration); z updated in place.  taus: host,
+ * n_taus >= 2, finite, every tau but the last > 0 (SFM_EINVAL otherwise).
+ * Uses no session and no weights.
+ */
+SFM_API int sfm_fm_solve_exact_velocity(const sfm_handle* h, const float* z0, float* z,
+                                        const float* taus, int n_taus, void* stream);
+
 /* ---- measurement ------------------------------------------------------------ */
 /* Kernel classes timed by the profiler (index into the arrays below). */
 #define SFM_PROF_APPEND     0   /* K/V cache append                          */

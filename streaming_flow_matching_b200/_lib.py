@@ -78,6 +78,7 @@ def _load():
         "sfm_linear": (i, [vp, vp, vp, i, i, i, i, i, vp]),
         "sfm_check_device_error": (i, [vp, C.POINTER(i)]),
         "sfm_euler_update": (i, [vp, vp, f, ll, vp]),
+        "sfm_fm_solve_exact_velocity": (i, [vp, vp, vp, C.POINTER(f), i, vp]),
         "sfm_profile_begin": (i, [i]),
         "sfm_profile_end": (i, [C.POINTER(C.c_double), C.POINTER(ll)]),
         "sfm_kernel_launch_count": (C.c_ulonglong, []),
@@ -99,7 +100,7 @@ EXPORTS = ["sfm_create", "sfm_destroy", "sfm_session_open", "sfm_session_reset",
            "sfm_session_get_info", "sfm_kvcache_append", "sfm_kvcache_read", "sfm_denoise_step",
            "sfm_fm_solve", "sfm_fm_solve_batched", "sfm_fm_solve_guided",
            "sfm_fm_solve_guided_batched", "sfm_set_graph_mode", "sfm_attention_workspace_bytes",
-           "sfm_attention", "sfm_attention_block_causal", "sfm_attention_noalloc", "sfm_linear", "sfm_euler_update", "sfm_profile_begin", "sfm_profile_end",
+           "sfm_attention", "sfm_attention_block_causal", "sfm_attention_noalloc", "sfm_linear", "sfm_euler_update", "sfm_fm_solve_exact_velocity", "sfm_profile_begin", "sfm_profile_end",
            "sfm_kernel_launch_count", "sfm_check_device_error", "sfm_strerror",
            "sfm_last_cuda_error"]
 

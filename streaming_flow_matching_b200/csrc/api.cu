@@ -806,6 +806,21 @@ int sfm_attention_block_causal(const void* q, const void* k, const void* v, void
                         workspace_bytes, (cudaStream_t)stream);
 }
 
+int sfm_fm_solve_exact_velocity(const sfm_handle* h, const float* z0, float* z, const float* taus,
+                                int n_taus, void* stream) {
+  if (!h || !z0 || !z) return SFM_EINVAL;
+  int rc = check_taus(taus, n_taus);
+  if (rc) return rc;
+  // the velocity (z - z0) / tau is evaluated at every tau but the last
+  for (int i = 0; i + 1 < n_taus; ++i)
+    if (!(taus[i] > 0.f)) return SFM_EINVAL;
+  const long long n = (long long)h->n_tok * h->cfg.c_lat;
+  for (int i = 0; i + 1 < n_taus; ++i)
+    if ((rc = launch_exact_velocity_euler(z, z0, taus[i], taus[i + 1], n, (cudaStream_t)stream)))
+      return rc;
+  return SFM_OK;
+}
+
 int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* stream) {
   if (n < 0 || (n > 0 && (!z || !v || !aligned16(z) || !aligned16(v))) || !isfinite(dtau))
     return SFM_EINVAL;

@@ -85,6 +85,8 @@ int launch_head_euler(const BatchDesc& b, const float* x, const void* g, const v
                       float eps, int dtype, cudaStream_t s, bool guided = false,
                       float scale = 1.f);
 int launch_euler(float* z, const float* v, float dtau, long long n, cudaStream_t s);
+int launch_exact_velocity_euler(float* z, const float* z0, float tau, float tau_next, long long n,
+                                cudaStream_t s);
 
 // GEMM C = A B^T, A [M][K], B [N][K] (both K-contiguous).
 enum Epilogue { EPI_F32 = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_STORE = 3, EPI_QKV = 4 };

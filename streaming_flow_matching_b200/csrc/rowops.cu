@@ -547,6 +547,31 @@ __global__ void euler_kernel(float* __restrict__ z, const float* __restrict__ v,
   if (t < n) z[t] = fmaf(dtau, v[t], z[t]);
 }
 
+// ---------------------------------------------------------------------------
+// exact-velocity Euler step (closed-form check of the solve loop): on the
+// rectified-flow path z_tau = (1 - tau) z0 + tau eps the velocity is
+// eps - z0 = (z_tau - z0) / tau, so a step evaluated at tau_i with that state-
+// dependent velocity stays on the path, and the solve ends at z0 for any schedule.
+// ---------------------------------------------------------------------------
+__global__ void exact_velocity_euler_kernel(float* __restrict__ z, const float* __restrict__ z0,
+                                            float inv_tau, float dtau, long long n) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const float zi = z[i];
+    const float v = (zi - z0[i]) * inv_tau;
+    z[i] = fmaf(dtau, v, zi);
+  }
+}
+
+int launch_exact_velocity_euler(float* z, const float* z0, float tau, float tau_next, long long n,
+                                cudaStream_t s) {
+  if (n <= 0) return SFM_OK;
+  long long blocks = (n + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  exact_velocity_euler_kernel<<<(unsigned)blocks, 256, 0, s>>>(z, z0, 1.f / tau, tau_next - tau, n);
+  return record_cuda(cudaGetLastError());
+}
+
 int launch_euler(float* z, const float* v, float dtau, long long n, cudaStream_t s) {
   if (n <= 0) return SFM_OK;
   int sms = 148;

@@ -166,6 +166,15 @@ class Performer:
         L.check(L.lib.sfm_fm_solve_guided_batched(self._h, n, s, u, zp, t, len(taus), scale, vp,
                                                   _stream()), "sfm_fm_solve_guided_batched")
 
+    def fm_solve_exact_velocity(self, z0, z, taus):
+        """Test-only: the Euler solve with the exact rectified-flow velocity (z - z0) / tau
+        in place of f_theta; from z = eps it ends at z0 for any schedule."""
+        _need(z0, torch.float32, "z0", (self.n_tok, self.shape["c_lat"]))
+        _need(z, torch.float32, "z", z0.shape)
+        t = (C.c_float * len(taus))(*taus)
+        L.check(L.lib.sfm_fm_solve_exact_velocity(self._h, _ptr(z0), _ptr(z), t, len(taus), _stream()),
+                "sfm_fm_solve_exact_velocity")
+
     def set_graph_mode(self, enabled):
         """Solves as one captured CUDA graph (True, the default) or direct launches."""
         L.check(L.lib.sfm_set_graph_mode(self._h, 1 if enabled else 0), "sfm_set_graph_mode")

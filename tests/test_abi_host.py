@@ -71,6 +71,7 @@ def test_null_arguments_are_rejected():
     assert L.lib.sfm_attention_block_causal(None, None, None, None, 4, 4, 2, 1, 128, 0, None, 0,
                                             None) == L.SFM_EINVAL
     taus = (C.c_float * 2)(1.0, 0.0)
+    assert L.lib.sfm_fm_solve_exact_velocity(None, None, None, taus, 2, None) == L.SFM_EINVAL
     assert L.lib.sfm_fm_solve_guided(None, 0, 1, None, taus, 2, 3.0, None) == L.SFM_EINVAL
     assert L.lib.sfm_fm_solve_guided_batched(None, 1, None, None, None, taus, 2, 3.0, None,
                                              None) == L.SFM_EINVAL

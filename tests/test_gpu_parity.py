@@ -244,3 +244,20 @@ def test_euler_exact_velocity_returns_clean_latent(cuda_device, n):
     euler_update(z, vel, -1.0)                       # one step 1 -> 0
     torch.cuda.synchronize()
     assert rel_l2(z.cpu().numpy(), z0.cpu().numpy()) <= 1e-6
+
+
+@pytest.mark.parametrize("taus", [[1.0, 0.75, 0.5, 0.25, 0.0], [1.0, 0.9, 0.3, 0.05, 0.0], [1.0, 0.0]],
+                         ids=["uniform4", "ragged4", "one-step"])
+def test_solve_loop_with_exact_velocity_returns_clean_latent(cuda_device, taus):
+    # the solve loop with f_theta replaced by the exact rectified-flow velocity
+    # (z - z0) / tau ends at z0 for any schedule (closed form); evaluating the
+    # velocity at a step's end point or stepping the wrong way would not
+    from streaming_flow_matching_b200 import Performer
+    w = S.TINY
+    p = Performer.from_workload(w, to_cuda(S.make_weights(w)), pool_tokens=w.n_tokens + w.unit_kv_tokens)
+    z0, eps = S.make_latents(w, device="cuda")
+    z = eps[0].clone()
+    p.fm_solve_exact_velocity(z0[0], z, taus)
+    torch.cuda.synchronize()
+    assert rel_l2(z.cpu().numpy(), z0[0].cpu().numpy()) <= 1e-6
+    p.close()

@@ -43,7 +43,11 @@ template <int BN, bool PAIR> struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int ACC_COLS = BN == 128 ? 128 : 256;     // TMEM columns between the two accumulators
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+  // after the stages: 256 B of barriers, then the epilogue's transpose buffers
+  // (4 warps x 32 rows x 32 fp32), then alignment slack
+  static constexpr int EPI_OFF = STAGES * STAGE_BYTES + 256;
+  static constexpr int EPI_BYTES = 4 * 32 * 32 * 4;
+  static constexpr int SMEM = EPI_OFF + EPI_BYTES + 1024;
 };
 
 __device__ __forceinline__ float gelu_tanh(float x) {
@@ -253,13 +257,28 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int m0 = (t % m_tiles) * TM + (int)rank * BM, n0 = (t / m_tiles) * BN;
       const int row = m0 + quarter * 32 + lane;
       const bool live = row < args.M;
-      // residual add: this row's fp32 slice of chunk 0 is loaded (from L2) while the
-      // tile's MMAs finish; chunk c + 1 while chunk c is read from TMEM and stored
+      // residual add, coalesced: the warp's 32 x 32 accumulator chunk goes through a
+      // shared-memory transpose, and lane (cg = lane & 7, rsub = lane >> 3) then handles
+      // float4 column group cg of rows 4 it + rsub (it = 0..7), so 8 lanes cover one
+      // row's 128 contiguous bytes.  The residual of chunk 0 is loaded (from L2) while
+      // the tile's MMAs finish; chunk c + 1 while chunk c is stored.
+      const int cg = lane & 7, rsub = lane >> 3;
+      const int wrow0 = m0 + quarter * 32;
       float4 res[2][8];
-      if (EPI == EPI_RESID && live) {
-        const float4* src = reinterpret_cast<const float4*>((const float*)args.C + (size_t)row * args.ldc + n0);
+      auto load_res = [&](int c, float4* dst) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) res[0][q] = src[q];
+        for (int it = 0; it < 8; ++it) {
+          const int rr = wrow0 + 4 * it + rsub;
+          if (rr < args.M)
+            dst[it] = *reinterpret_cast<const float4*>((const float*)args.C + (size_t)rr * args.ldc + n0 +
+                                                       c * 32 + cg * 4);
+        }
+      };
+      if (EPI == EPI_RESID) {
+        // the epilogue warps idle through the mainloop: pull this row's residual slice
+        // into L2 now (it was written several kernels ago and may have left L2)
+        if (live) prefetch_l2_bulk((const float*)args.C + (size_t)row * args.ldc + n0, BN * 4);
+        load_res(0, res[0]);
       }
       // fused RMSNorm of the A rows: 1 / rms of this row from the producer's partial sums
       float rinv = 1.f;
@@ -323,56 +342,67 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       } else if (EPI == EPI_RESID) {
-        float ssq = 0.f;
+        float4* stg = reinterpret_cast<float4*>(smem + C::EPI_OFF) + quarter * (32 * 8);
+        float ssq[8];
+#pragma unroll
+        for (int it = 0; it < 8; ++it) ssq[it] = 0.f;
         // unrolled so the two residual buffers stay in registers
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
-          if (live && c + 1 < BN / 32) {
-            const float4* src = reinterpret_cast<const float4*>((const float*)args.C + (size_t)row * args.ldc +
-                                                                n0 + (c + 1) * 32);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) res[(c + 1) & 1][q] = src[q];
-          }
+          if (c + 1 < BN / 32) load_res(c + 1, res[(c + 1) & 1]);
           uint32_t r[32];
           tmem_ld32(tbase + c * 32, r);
           tmem_wait_ld(r);
-          if (!live) continue;
-          float4* d = reinterpret_cast<float4*>((float*)args.C + (size_t)row * args.ldc + n0 + c * 32);
-          float xs[32];
+          // row `lane` of the chunk; float4 slot k stored at k ^ (lane & 7) (no bank conflicts)
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 x = res[c & 1][q];
-            x.x += __uint_as_float(r[4 * q]);
-            x.y += __uint_as_float(r[4 * q + 1]);
-            x.z += __uint_as_float(r[4 * q + 2]);
-            x.w += __uint_as_float(r[4 * q + 3]);
-            d[q] = x;
-            xs[4 * q] = x.x;
-            xs[4 * q + 1] = x.y;
-            xs[4 * q + 2] = x.z;
-            xs[4 * q + 3] = x.w;
-          }
+          for (int k = 0; k < 8; ++k)
+            stg[lane * 8 + (k ^ (lane & 7))] =
+                make_float4(__uint_as_float(r[4 * k]), __uint_as_float(r[4 * k + 1]),
+                            __uint_as_float(r[4 * k + 2]), __uint_as_float(r[4 * k + 3]));
+          __syncwarp();
+          const int col = n0 + c * 32 + cg * 4;
+          float gv[4] = {1.f, 1.f, 1.f, 1.f};
           if (args.g_next) {
-            // the next RMSNorm's numerator bf16(x g) and this row's sum of squares
-            const uint4* g4 = reinterpret_cast<const uint4*>(args.g_next + n0 + c * 32);
+            const uint2 gu = __ldg(reinterpret_cast<const uint2*>(args.g_next + col));
+            const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gu.x));
+            const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&gu.y));
+            gv[0] = g01.x; gv[1] = g01.y; gv[2] = g23.x; gv[3] = g23.y;
+          }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 gu = __ldg(g4 + q);
-              const __nv_bfloat162* gh = reinterpret_cast<const __nv_bfloat162*>(&gu);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 gf = __bfloat1622float2(gh[e]);
-                const int i = 8 * q + 2 * e;
-                ssq = fmaf(xs[i], xs[i], ssq);
-                ssq = fmaf(xs[i + 1], xs[i + 1], ssq);
-                xs[i] *= gf.x;
-                xs[i + 1] *= gf.y;
-              }
+          for (int it = 0; it < 8; ++it) {
+            const int rl = 4 * it + rsub;
+            const int rr = wrow0 + rl;
+            const float4 a = stg[rl * 8 + (cg ^ (rl & 7))];
+            if (rr >= args.M) continue;
+            float4 x = res[c & 1][it];
+            x.x += a.x;
+            x.y += a.y;
+            x.z += a.z;
+            x.w += a.w;
+            *reinterpret_cast<float4*>((float*)args.C + (size_t)rr * args.ldc + col) = x;
+            if (args.g_next) {
+              // the next RMSNorm's numerator bf16(x g) and this row's sum of squares
+              ssq[it] = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, ssq[it]))));
+              uint2 o;
+              o.x = pack_bf16x2(x.x * gv[0], x.y * gv[1]);
+              o.y = pack_bf16x2(x.z * gv[2], x.w * gv[3]);
+              *reinterpret_cast<uint2*>(args.xg + (size_t)rr * args.ldc + col) = o;
             }
-            store_bf16x32(args.xg + (size_t)row * args.ldc + n0 + c * 32, xs);
+          }
+          __syncwarp();   // the next chunk overwrites the transpose buffer
+        }
+        if (args.g_next) {
+          // each row's partial sum over this tile: the 8 lanes of its column groups
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            float t = ssq[it];
+            t += __shfl_xor_sync(0xffffffffu, t, 1);
+            t += __shfl_xor_sync(0xffffffffu, t, 2);
+            t += __shfl_xor_sync(0xffffffffu, t, 4);
+            const int rr = wrow0 + 4 * it + rsub;
+            if (cg == 0 && rr < args.M) args.ss_out[(size_t)rr * args.ss_ld + n0 / BN] = t;
           }
         }
-        if (args.g_next && live) args.ss_out[(size_t)row * args.ss_ld + n0 / BN] = ssq;
       } else {
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];

@@ -89,6 +89,16 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
 }
+
+// Bulk prefetch of `bytes` (a multiple of 16) from global memory at a 16-byte
+// aligned address into L2; a hint with no completion to wait for.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .u64 ga;\n\tcvta.to.global.u64 ga, %0;\n\t"
+      "cp.async.bulk.prefetch.L2.global [ga], %1;\n\t}" ::"l"(p),
+      "r"(bytes)
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1) {
   asm volatile(

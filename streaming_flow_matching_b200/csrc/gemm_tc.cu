@@ -498,9 +498,12 @@ bool gemm_tc_pair(int M, int N, int hd, int epi, int sms) {
 }
 
 int gemm_tc_block_n(int M, int N, int hd, int epi, int sms, bool pair) {
-  // N-tile width minimising (waves of the persistent grid) x (work per tile);
-  // ties go to the wider tile.  The QKV epilogue works on whole 128-wide heads.
-  // Pairs take 256-row tiles and run on sms / 2 units.
+  // N-tile width minimising (waves of the persistent grid) x (time per tile); ties
+  // go to the wider tile.  A tile's time is modelled as BN + 128 columns: a k-block's
+  // time is set mostly by the round trip of its operand stages, not by BN (measured
+  // per k-block on 924 / 7392-row projections: ~680 cycles for 256-wide pair tiles,
+  // ~626 for 128-wide ones), so narrow tiles cost more per column.  The QKV epilogue
+  // works on whole 128-wide heads.  Pairs take 256-row tiles and run on sms / 2 units.
   const int cands[3] = {256, 192, 128};
   if (pair) sms /= 2;
   const int tm = pair ? 2 * gtc::BM : gtc::BM;
@@ -511,7 +514,7 @@ int gemm_tc_block_n(int M, int N, int hd, int epi, int sms, bool pair) {
     if (N % bn) continue;
     if (epi == EPI_QKV && (bn % 128 || hd % bn)) continue;
     const long long tiles = m_tiles * (N / bn);
-    const long long cost = ((tiles + sms - 1) / sms) * bn;
+    const long long cost = ((tiles + sms - 1) / sms) * (bn + 128);
     if (!best || cost < best_cost) {
       best = bn;
       best_cost = cost;

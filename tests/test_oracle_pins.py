@@ -153,6 +153,26 @@ def test_block_causal_mask():
     np.testing.assert_allclose(out[:2], O.attention(q[:2], k[:2], v[:2]), atol=1e-15)
 
 
+def test_masked_attention_with_prefix_brute_force():
+    # the form a multi-unit pass uses: prefix keys in unit -1 (visible to every query),
+    # then the queries' own keys in units of uneven length; each row against the
+    # scalar-loop attention over exactly the keys it may see
+    q_units = [0, 0, 0, 1, 1, 2]
+    k_units = [-1, -1] + q_units
+    vis = O.block_causal_visible(q_units, k_units)
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((6, 2, 4))
+    k = rng.standard_normal((8, 2, 4))
+    v = rng.standard_normal((8, 2, 4))
+    out = O.attention(q, k, v, vis)
+    for i in range(6):
+        seen = [j for j in range(8) if k_units[j] <= q_units[i]]
+        assert len(seen) == 2 + sum(1 for u in q_units if u <= q_units[i])
+        for h in range(2):
+            ref = BF.attend(list(q[i, h]), [list(k[j, h]) for j in seen], [list(v[j, h]) for j in seen])
+            np.testing.assert_allclose(out[i, h], ref, atol=1e-14)
+
+
 # --------------------------------------------------------------------------
 # RMSNorm, RoPE, GELU, tau embedding, linear
 # --------------------------------------------------------------------------

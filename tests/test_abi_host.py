@@ -26,7 +26,11 @@ def test_every_declared_symbol_is_exported():
     lib = C.CDLL(L.LIB_PATH)
     missing = [n for n in names if not hasattr(lib, n)]
     assert not missing, missing
-    assert set(L.EXPORTS) <= set(names)
+    # the binding covers exactly the declared calls, each with a declared signature
+    assert sorted(L.EXPORTS) == sorted(names)
+    assert len(set(names)) == len(names)
+    for n in names:
+        assert getattr(L.lib, n).argtypes is not None, n
 
 
 def cfg(**kw):

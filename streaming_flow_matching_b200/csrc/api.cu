@@ -245,9 +245,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
     return g;
   };
   const AttnDesc ad = attn_desc(b);
-  long long max_keys = 0;
-  for (int i = 0; i < b.n; ++i) max_keys = ad.nkeys[i] > max_keys ? ad.nkeys[i] : max_keys;
-  const int splits = tc ? attention_tc_splits(b.n_tok, b.n, max_keys, c.n_heads, h->sms) : 1;
+  const int splits = tc ? attention_tc_splits_batch(ad, c.n_heads, h->sms) : 1;
   for (int l = 0; l < c.n_layers; ++l) {
     if (!tc) {
       ProfScope ps(SFM_PROF_ROWOPS, s);

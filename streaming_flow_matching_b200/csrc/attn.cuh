@@ -47,6 +47,8 @@ int launch_attention_merge(const float* o_part, const float* lse_part, void* o,
 // unit_rows > 0: block-causal (see AttnDesc), which shortens the early query blocks.
 int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads,
                         int sms, int unit_rows = 0);
+// A batch whose sessions have their own key counts (AttnDesc::nkeys).
+int attention_tc_splits_batch(const AttnDesc& a, int n_heads, int sms);
 // mq: map over the query rows [rows][H][128]; mk, mv: maps over the key rows, of
 // which this call uses rows kv_row0 + kbase[s] + [0, nkeys[s]).
 int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,

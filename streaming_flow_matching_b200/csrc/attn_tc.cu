@@ -516,40 +516,71 @@ __global__ void __launch_bounds__(THREADS, 1)
 //   merge     = its bytes (fp32 partials of every split read, bf16 O written) / kMergeBps.
 // More splits fill the SMs and shorten the longest CTA; each split adds fixed cost and
 // merge traffic.  Block-causal calls count each query block's own key tiles.
-int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads,
-                        int sms, int unit_rows) {
+namespace {
+
+// key tiles of query block b of a session with `keys` keys
+long long block_tiles(int rows_per, long long keys, int unit_rows, int b) {
+  const int last = (b + 1) * atc::ROWS < rows_per ? (b + 1) * atc::ROWS - 1 : rows_per - 1;
+  const long long lim = unit_rows > 0 && keys < (1LL << 31)
+                            ? attn_key_limit((int)keys, rows_per, unit_rows, last)
+                            : keys;
+  return (lim + atc::BKV - 1) / atc::BKV;
+}
+
+// Split count from a cost model of the kernel, in microseconds on a B200:
+//   CTA time  = (key tiles of the CTA) x kStepUs + kCtaUs (set-up, output, hand-over),
+//   kernel    = max(waves x mean CTA time, longest CTA time), waves = ceil(CTAs / SMs),
+//   merge     = its bytes (fp32 partials of every split read, bf16 O written) / kMergeBps.
+// More splits fill the SMs and shorten the longest CTA; each split adds fixed cost and
+// merge traffic.  tiles_of(i): key tiles of query block i (i < n_blocks); every block
+// runs n_heads CTAs per split; merge_rows = query rows x heads.
+template <typename F>
+int choose_splits(F tiles_of, int n_blocks, int n_heads, double merge_rows, int sms) {
   constexpr double kStepUs = 2.0, kCtaUs = 5.0, kMergeBps = 4.0e6;   // bytes per microsecond
-  const int qtiles = (rows_per_session + atc::ROWS - 1) / atc::ROWS;
-  const long long ctas = (long long)n_sessions * qtiles * n_heads;
-  const long long tiles = (max_keys + atc::BKV - 1) / atc::BKV;
+  long long max_tiles = 0;
+  for (int i = 0; i < n_blocks; ++i) max_tiles = tiles_of(i) > max_tiles ? tiles_of(i) : max_tiles;
+  const long long ctas = (long long)n_blocks * n_heads;
   int best = 1;
   double best_us = 0.0;
   for (int s = 1; s <= kMaxSplits; ++s) {
-    if (s > 1 && tiles / s < 2) break;
+    if (s > 1 && max_tiles / s < 2) break;
     double sum_t = 0.0, max_t = 0.0;
-    for (int b = 0; b < qtiles; ++b) {
-      const int last = (b + 1) * atc::ROWS < rows_per_session ? (b + 1) * atc::ROWS - 1 : rows_per_session - 1;
-      const long long lim = unit_rows > 0 && max_keys < (1LL << 31)
-                                ? attn_key_limit((int)max_keys, rows_per_session, unit_rows, last)
-                                : max_keys;
-      const double t = (double)(((lim + atc::BKV - 1) / atc::BKV + s - 1) / s) * kStepUs + kCtaUs;
+    for (int i = 0; i < n_blocks; ++i) {
+      const double t = (double)((tiles_of(i) + s - 1) / s) * kStepUs + kCtaUs;
       sum_t += t;
       max_t = t > max_t ? t : max_t;
     }
     const long long work = ctas * s;
     const double waves = (double)((work + sms - 1) / sms);
-    double us = waves * sum_t / qtiles;
+    double us = waves * sum_t / n_blocks;
     if (max_t > us) us = max_t;
-    if (s > 1) {
-      const double rows = (double)n_sessions * rows_per_session * n_heads;
-      us += (s * rows * (atc::D + 1) * 4.0 + rows * atc::D * 2.0) / kMergeBps;
-    }
+    if (s > 1) us += (s * merge_rows * (atc::D + 1) * 4.0 + merge_rows * atc::D * 2.0) / kMergeBps;
     if (s == 1 || us < best_us) {
       best = s;
       best_us = us;
     }
   }
   return best;
+}
+
+}  // namespace
+
+// n_sessions identical sessions of max_keys keys; block-causal calls (unit_rows > 0)
+// count each query block's own key tiles.
+int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads,
+                        int sms, int unit_rows) {
+  const int qtiles = (rows_per_session + atc::ROWS - 1) / atc::ROWS;
+  return choose_splits(
+      [&](int i) { return block_tiles(rows_per_session, max_keys, unit_rows, i % qtiles); },
+      n_sessions * qtiles, n_heads, (double)n_sessions * rows_per_session * n_heads, sms);
+}
+
+// A batch whose sessions have their own key counts (ragged caches).
+int attention_tc_splits_batch(const AttnDesc& a, int n_heads, int sms) {
+  const int qtiles = (a.rows_per + atc::ROWS - 1) / atc::ROWS;
+  return choose_splits(
+      [&](int i) { return block_tiles(a.rows_per, a.nkeys[i / qtiles], a.unit_rows, i % qtiles); },
+      a.n * qtiles, n_heads, (double)a.n * a.rows_per * n_heads, sms);
 }
 
 // q: map over [rows][H][128]; k, v: maps over the key rows ([rows][H][128]).

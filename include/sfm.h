@@ -179,8 +179,9 @@ SFM_API int sfm_fm_solve(sfm_handle* h, int session, float* z, const float* taus
                  int n_taus, void* stream);
 
 /* Batched solve over n_sessions open sessions (distinct ids), each with its
- * own cache length; z[i] is session i's device fp32 [N][C].  sessions and z
- * are host arrays.  SFM_ECAPACITY if n_sessions > max_sessions. */
+ * own cache length; z[i] is session i's device fp32 [N][C] (distinct buffers:
+ * SFM_EINVAL if two entries are the same pointer).  sessions and z are host
+ * arrays.  SFM_ECAPACITY if n_sessions > max_sessions. */
 SFM_API int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions,
                          float* const* z, const float* taus, int n_taus, void* stream);
 
@@ -210,9 +211,10 @@ SFM_API int sfm_fm_solve_guided(sfm_handle* h, int session, int uncond_session, 
 /*
  * n_pairs guided solves in one batch of 2 * n_pairs evaluations.  sessions,
  * uncond_sessions, z: host arrays of n_pairs entries (z[p] device fp32
- * [N][C]); all 2 * n_pairs session ids distinct.  v_out: NULL, or a host
- * array of n_pairs device fp32 [N][C] buffers (entries may be NULL) that
- * receive the guided velocity of the last step.  SFM_ECAPACITY if
+ * [N][C], distinct buffers); all 2 * n_pairs session ids distinct.  v_out:
+ * NULL, or a host array of n_pairs device fp32 [N][C] buffers (entries may be
+ * NULL; non-NULL ones distinct) that receive the guided velocity of the last
+ * step.  SFM_EINVAL if a z or v_out buffer repeats.  SFM_ECAPACITY if
  * 2 * n_pairs > max_sessions.
  */
 SFM_API int sfm_fm_solve_guided_batched(sfm_handle* h, int n_pairs, const int* sessions,

@@ -682,11 +682,13 @@ int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions, flo
   if (!h->has_weights) return SFM_EINVAL;
   if (n_sessions > h->cfg.max_sessions) return SFM_ECAPACITY;
   int rc;
+  // distinct sessions (each writes its unit's K/V into its own scratch rows) and
+  // distinct latents (each session's Euler update writes its own z)
   for (int i = 0; i < n_sessions; ++i) {
     if ((rc = session_ok(h, sessions[i]))) return rc;
     if (!z[i]) return SFM_EINVAL;
     for (int j = 0; j < i; ++j)
-      if (sessions[j] == sessions[i]) return SFM_EINVAL;
+      if (sessions[j] == sessions[i] || z[j] == z[i]) return SFM_EINVAL;
   }
   if ((rc = check_taus(taus, n_taus))) return rc;
   return solve(h, n_sessions, sessions, z, taus, n_taus, nullptr, (cudaStream_t)stream);
@@ -704,6 +706,9 @@ int sfm_fm_solve_guided_batched(sfm_handle* h, int n_pairs, const int* sessions,
   float* vs[kMaxBatch];
   for (int p = 0; p < n_pairs; ++p) {
     if (!z[p]) return SFM_EINVAL;
+    // each pair's Euler update writes its own z and velocity
+    for (int q = 0; q < p; ++q)
+      if (z[q] == z[p] || (v_out && v_out[p] && v_out[q] == v_out[p])) return SFM_EINVAL;
     ids[2 * p] = sessions[p];
     ids[2 * p + 1] = uncond_sessions[p];
     zs[2 * p] = zs[2 * p + 1] = z[p];

@@ -82,4 +82,8 @@ def test_batched_argument_errors(cuda_device):
     arr = (C.c_int * 1)(sessions[0])
     zp = (C.c_void_p * 1)(z[0].data_ptr())
     assert L.lib.sfm_fm_solve_batched(p._h, 1, arr, zp, bad, 1, st) == L.SFM_EINVAL  # one tau
+    # the same latent buffer for two sessions: both Euler updates would write it
+    arr2 = (C.c_int * 2)(sessions[0], sessions[1])
+    zsame = (C.c_void_p * 2)(z[0].data_ptr(), z[0].data_ptr())
+    assert L.lib.sfm_fm_solve_batched(p._h, 2, arr2, zsame, taus, 3, st) == L.SFM_EINVAL
     p.close()

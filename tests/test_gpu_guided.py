@@ -150,6 +150,13 @@ def test_guided_argument_errors(cuda_device):
         p.fm_solve_guided_batched([s, u], [u, s], [z, z.clone()], taus, 2.0)
     assert e.value.status == L.SFM_ECAPACITY
     p.close()
+    # two pairs sharing one latent buffer: both Euler updates would write it
+    p4 = _performer(w, weights, [2, 1, 2, 1])
+    ids = [p4.open_session(c) for c in (2, 1, 2, 1)]
+    with pytest.raises(L.SfmError) as e:
+        p4.fm_solve_guided_batched(ids[0::2], ids[1::2], [z, z], taus, 2.0)
+    assert e.value.status == L.SFM_EINVAL
+    p4.close()
     # one session per handle: no room for the unconditional evaluation
     p1 = _performer(w, weights, [2])
     s1 = p1.open_session(2)

@@ -164,7 +164,8 @@ SFM_API int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long l
  * One Euler step of the current unit: v = f_theta(z, tau_from | cache),
  * z <- z + (tau_to - tau_from) v.  z: device fp32 [N][C], N = n_video +
  * n_audio (video rows first), updated in place.  v_out: nullable device fp32
- * [N][C] receiving v.  The current unit's tokens are at positions p0 + j.
+ * [N][C] receiving v, a buffer other than z (SFM_EINVAL otherwise).  The
+ * current unit's tokens are at positions p0 + j.
  */
 SFM_API int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_from,
                      float tau_to, float* v_out, void* stream);
@@ -213,8 +214,8 @@ SFM_API int sfm_fm_solve_guided(sfm_handle* h, int session, int uncond_session, 
  * uncond_sessions, z: host arrays of n_pairs entries (z[p] device fp32
  * [N][C], distinct buffers); all 2 * n_pairs session ids distinct.  v_out:
  * NULL, or a host array of n_pairs device fp32 [N][C] buffers (entries may be
- * NULL; non-NULL ones distinct) that receive the guided velocity of the last
- * step.  SFM_EINVAL if a z or v_out buffer repeats.  SFM_ECAPACITY if
+ * NULL; non-NULL ones distinct, none of them a z) that receive the guided
+ * velocity of the last step.  SFM_EINVAL if a z or v_out buffer repeats.  SFM_ECAPACITY if
  * 2 * n_pairs > max_sessions.
  */
 SFM_API int sfm_fm_solve_guided_batched(sfm_handle* h, int n_pairs, const int* sessions,

@@ -660,6 +660,7 @@ int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_from, float
   int rc = session_ok(h, session);
   if (rc) return rc;
   if (!h->has_weights || !z || !isfinite(tau_from) || !isfinite(tau_to)) return SFM_EINVAL;
+  if (v_out == z) return SFM_EINVAL;   // the step writes both
   const float taus[2] = {tau_from, tau_to};
   float* zs[1] = {z};
   float* vs[1] = {v_out};
@@ -707,8 +708,10 @@ int sfm_fm_solve_guided_batched(sfm_handle* h, int n_pairs, const int* sessions,
   for (int p = 0; p < n_pairs; ++p) {
     if (!z[p]) return SFM_EINVAL;
     // each pair's Euler update writes its own z and velocity
-    for (int q = 0; q < p; ++q)
-      if (z[q] == z[p] || (v_out && v_out[p] && v_out[q] == v_out[p])) return SFM_EINVAL;
+    for (int q = 0; q < n_pairs; ++q) {
+      if (q < p && (z[q] == z[p] || (v_out && v_out[p] && v_out[q] == v_out[p]))) return SFM_EINVAL;
+      if (v_out && v_out[p] && v_out[p] == z[q]) return SFM_EINVAL;
+    }
     ids[2 * p] = sessions[p];
     ids[2 * p + 1] = uncond_sessions[p];
     zs[2 * p] = zs[2 * p + 1] = z[p];

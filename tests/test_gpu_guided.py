@@ -156,6 +156,13 @@ def test_guided_argument_errors(cuda_device):
     with pytest.raises(L.SfmError) as e:
         p4.fm_solve_guided_batched(ids[0::2], ids[1::2], [z, z], taus, 2.0)
     assert e.value.status == L.SFM_EINVAL
+    z2 = z.clone()
+    with pytest.raises(L.SfmError) as e:                # a velocity output that is a latent
+        p4.fm_solve_guided_batched(ids[0::2], ids[1::2], [z, z2], taus, 2.0, v_outs=[z2, None])
+    assert e.value.status == L.SFM_EINVAL
+    with pytest.raises(L.SfmError) as e:
+        p4.denoise_step(ids[0], z, 1.0, 0.5, z)
+    assert e.value.status == L.SFM_EINVAL
     p4.close()
     # one session per handle: no room for the unconditional evaluation
     p1 = _performer(w, weights, [2])

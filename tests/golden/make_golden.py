@@ -10,6 +10,9 @@ import sfm_synth as S                      # noqa: E402
 from oracle import sfm_oracle as O         # noqa: E402
 
 
+GUIDED_SCALE = 3.5
+
+
 def tiny_case():
     w = S.TINY
     cfg = O.Config(w.n_layers, w.d_model, w.n_heads, w.head_dim, w.d_mlp, w.c_lat,
@@ -29,7 +32,13 @@ def main():
                     cache.tokens_appended)
     z = O.denoise_solve(cfg, eps, taus, weights, cache.k, cache.v, cache.valid_tokens,
                         cache.tokens_appended)
+    # classifier-free guidance against an empty unconditional context
+    empty = [O.f64(cache.k[0][:0])] * w.n_layers
+    zg = O.denoise_solve_cfg(cfg, eps, taus, weights,
+                             (cache.k, cache.v, cache.valid_tokens, cache.tokens_appended),
+                             (empty, empty, 0, 0), GUIDED_SCALE)
     out = {"workload": w.name, "taus": taus,
+           "guided_scale": GUIDED_SCALE, "guided_solve_rows0to3": zg[:4].tolist(),
            "velocity_tau1_rows0to3": vel[:4].tolist(),
            "solve_rows0to3": z[:4].tolist(),
            "velocity_tau1_l2": float((vel ** 2).sum() ** 0.5),

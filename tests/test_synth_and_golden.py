@@ -58,3 +58,8 @@ def test_oracle_reproduces_committed_regression_fixture():
     z = O.denoise_solve(cfg, eps, gold["taus"], weights, cache.k, cache.v, cache.valid_tokens,
                         cache.tokens_appended)
     np.testing.assert_allclose(z[:4], np.array(gold["solve_rows0to3"]), rtol=1e-12, atol=1e-13)
+    empty = [O.f64(cache.k[0][:0])] * w.n_layers
+    zg = O.denoise_solve_cfg(cfg, eps, gold["taus"], weights,
+                             (cache.k, cache.v, cache.valid_tokens, cache.tokens_appended),
+                             (empty, empty, 0, 0), gold["guided_scale"])
+    np.testing.assert_allclose(zg[:4], np.array(gold["guided_solve_rows0to3"]), rtol=1e-12, atol=1e-13)

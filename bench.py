@@ -152,19 +152,28 @@ def append_bytes(w):
     return 2 * 2 * w.n_layers * w.unit_kv_tokens * w.hd * 2   # K and V, read + write, bf16
 
 
-def source_hash(path):
+KERNEL_END = b"}  // namespace atc\n"   # the attention source's device code ends here
+
+
+def kernel_hash(path):
+    """sha256 (16 hex digits) of a kernel source's device code: the text up to the end of
+    its kernel namespace (host-side launch and planning code after it does not change the
+    kernel's memory traffic)."""
     with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+        src = f.read()
+    end = src.find(KERNEL_END)
+    return hashlib.sha256(src if end < 0 else src[:end + len(KERNEL_END)]).hexdigest()[:16]
 
 
-def traffic_for(kernel_src):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this source."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+def traffic_for(kernel_src, table=None):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel
+    code; None otherwise."""
+    path = table or os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
         ent = t[os.path.basename(kernel_src)]
-        if ent["source_sha256_16"] != source_hash(kernel_src):
+        if ent["kernel_sha256_16"] != kernel_hash(kernel_src):
             return None
         return ent["dram_bytes_per_launch"]
     except Exception:

@@ -33,3 +33,19 @@ def test_kernel_edits_drop_the_record(tmp_path):
     assert end > 0
     p = _copy(tmp_path, lambda t: t[:end] + b"// changed\n" + t[end:])
     assert bench.traffic_for(p, TABLE) is None
+
+
+def test_roofline_work_counts_at_640x368():
+    # the numerators of the bench's roofline fractions, against hand counts:
+    # attention 4 N (S_c + N) H D per layer launch, GEMMs 2 M K N, append K+V read + write
+    import sfm_synth as S
+    w = S.V02
+    fl = bench.flop_counts(w, [57600])
+    assert fl["attention_per_launch"] == 4 * 924 * (57600 + 924) * 24 * 128 == 664488050688
+    assert fl["gemm_per_layer"] == 2 * 924 * 3072 * (9216 + 3072 + 12288 + 12288)
+    assert abs(fl["per_euler_step"] / 1e12 - 24.47) < 0.01
+    assert bench.append_bytes(w) == 2 * 2 * 28 * 1200 * 3072 * 2 == 825753600
+    # a ragged batch counts every session's own cache
+    fl2 = bench.flop_counts(w, [57600, 1200])
+    assert fl2["attention_per_launch"] == fl["attention_per_launch"] + 4 * 924 * (1200 + 924) * 3072
+    assert fl2["gemm_per_layer"] == 2 * fl["gemm_per_layer"]

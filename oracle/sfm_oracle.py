@@ -21,7 +21,7 @@ Sources (the pages are web write-ups of Wan-Streamer; none prints code):
   [blog]  "Wan-Streamer v0.2" blog (zhao9797.github.io): "Infra" section.
   [abs]   "Wan-Streamer v0.2" abstract (chatpaper.ai).
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * rectified-flow path z_tau = (1 - tau) z0 + tau eps, velocity eps - z0
     (the path formula of [v0.1] §3.4 was lost in extraction; the symbol glosses
     survive); Euler solve from tau = 1 to tau = 0, z <- z + (tau_next - tau) v.
@@ -384,6 +384,38 @@ def f_theta_sequence(cfg: Config, zs, taus, w, return_kv=False):
     empty = np.zeros((0, cfg.n_heads, cfg.head_dim))
     for lw in w["layers"]:
         x, k, v = layer_forward(cfg, x, lw, empty, empty, pos, visible, return_kv=True)
+        kv.append((k, v))
+    vel = head(cfg, x, w)
+    out = [vel[u * n:(u + 1) * n] for u in range(n_units)]
+    if return_kv:
+        return out, kv
+    return out
+
+
+def f_theta_units(cfg: Config, zs, taus, w, cache_k, cache_v, valid_tokens, p0, return_kv=False):
+    """Several consecutive units after a clean cached prefix, in one masked pass.
+
+    [v0.1] §3.3: a unit sees itself bidirectionally and every earlier unit, never a
+    later one; the cached prefix (the clean context of §3.4) counts as earlier than
+    every unit of the pass.  Unit u's tokens sit at positions p0 + u * N + j (the
+    units follow the cache on the timeline).  zs, taus: per-unit latents [N][C] and
+    flow times.  cache_k / cache_v: per-layer [rows][H][D], first valid_tokens rows
+    valid (already rotated).  Returns the per-unit velocities and, optionally,
+    every layer's rotated K/V of the pass's own tokens.  One unit is f_theta; an
+    empty prefix with p0 = 0 is f_theta_sequence.
+    """
+    n = cfg.n_tokens
+    n_units = len(zs)
+    x = np.concatenate([embed(cfg, zs[u], taus[u], w) for u in range(n_units)], axis=0)
+    units = np.repeat(np.arange(n_units), n)
+    pos = p0 + np.arange(n_units * n)
+    key_units = np.concatenate([np.full(valid_tokens, -1), units])   # prefix = unit -1
+    visible = block_causal_visible(units, key_units)
+    kv = []
+    for li, lw in enumerate(w["layers"]):
+        kc = f64(cache_k[li][:valid_tokens])
+        vc = f64(cache_v[li][:valid_tokens])
+        x, k, v = layer_forward(cfg, x, lw, kc, vc, pos, visible, return_kv=True)
         kv.append((k, v))
     vel = head(cfg, x, w)
     out = [vel[u * n:(u + 1) * n] for u in range(n_units)]

@@ -378,6 +378,66 @@ def test_performer_form_equals_block_causal_sequence():
     np.testing.assert_allclose(got, seq[-1], atol=1e-12)
 
 
+def _units_problem(seed, n_units=3, S=10):
+    cfg = tiny_cfg(unit_kv_tokens=5)
+    rng = np.random.default_rng(seed)
+    w = tiny_weights(cfg, rng)
+    ck = [rng.standard_normal((S + 4, cfg.n_heads, cfg.head_dim)) for _ in range(cfg.n_layers)]
+    cv = [rng.standard_normal((S + 4, cfg.n_heads, cfg.head_dim)) for _ in range(cfg.n_layers)]
+    zs = [rng.standard_normal((cfg.n_tokens, cfg.c_lat)) for _ in range(n_units)]
+    return cfg, w, ck, cv, zs, S
+
+
+def test_units_pass_with_empty_prefix_is_the_block_causal_sequence():
+    cfg, w, ck, cv, zs, _ = _units_problem(40)
+    taus = [0.0, 0.3, 1.0]
+    seq, kv_seq = O.f_theta_sequence(cfg, zs, taus, w, return_kv=True)
+    got, kv = O.f_theta_units(cfg, zs, taus, w, ck, cv, 0, 0, return_kv=True)
+    for a, b in zip(got, seq):
+        np.testing.assert_allclose(a, b, atol=1e-12)
+    for (k1, v1), (k2, v2) in zip(kv, kv_seq):
+        np.testing.assert_allclose(k1, k2, atol=1e-12)
+        np.testing.assert_allclose(v1, v2, atol=1e-12)
+
+
+def test_units_pass_of_one_unit_is_f_theta():
+    cfg, w, ck, cv, zs, S = _units_problem(41, n_units=1)
+    got = O.f_theta_units(cfg, zs, [0.7], w, ck, cv, S, 37)[0]
+    np.testing.assert_allclose(got, O.f_theta(cfg, zs[0], 0.7, w, ck, cv, S, 37), atol=1e-12)
+    # and the brute-force scalar loops agree
+    np.testing.assert_allclose(got, np.array(BF.velocity(cfg, zs[0], 0.7, w, ck, cv, S, 37)),
+                               rtol=1e-11, atol=1e-12)
+
+
+def test_units_pass_equals_performer_form_over_the_grown_cache():
+    # unit u of the pass sees the prefix and units < u: the performer form with those
+    # units' own K/V appended to the cache (positions continuing) gives the same result
+    cfg, w, ck, cv, zs, S = _units_problem(42, n_units=3)
+    taus = [0.0, 0.25, 0.9]
+    p0 = 19
+    got, kv = O.f_theta_units(cfg, zs, taus, w, ck, cv, S, p0, return_kv=True)
+    n = cfg.n_tokens
+    for u in range(3):
+        gk = [np.concatenate([ck[l][:S], kv[l][0][:u * n]]) for l in range(cfg.n_layers)]
+        gv = [np.concatenate([cv[l][:S], kv[l][1][:u * n]]) for l in range(cfg.n_layers)]
+        ref = O.f_theta(cfg, zs[u], taus[u], w, gk, gv, S + u * n, p0 + u * n)
+        np.testing.assert_allclose(got[u], ref, atol=1e-12)
+
+
+def test_units_pass_later_units_do_not_leak_and_prefix_matters():
+    cfg, w, ck, cv, zs, S = _units_problem(43, n_units=3)
+    taus = [0.5, 0.5, 0.5]
+    base = O.f_theta_units(cfg, zs, taus, w, ck, cv, S, 3)
+    zs2 = list(zs); zs2[2] = zs[2] + 4.0
+    pert = O.f_theta_units(cfg, zs2, taus, w, ck, cv, S, 3)
+    assert np.array_equal(base[0], pert[0]) and np.array_equal(base[1], pert[1])
+    assert not np.array_equal(base[2], pert[2])
+    ck2 = [c.copy() for c in ck]
+    ck2[1][0] += 1.0                                  # a cached key every unit sees
+    moved = O.f_theta_units(cfg, zs, taus, w, ck2, cv, S, 3)
+    assert all(np.max(np.abs(m - b)) > 1e-9 for m, b in zip(moved, base))
+
+
 def test_solve_with_network_is_euler_over_f_theta():
     cfg, w, ck, cv, z, S = _tiny_problem(19)
     taus = [1.0, 0.5, 0.0]

@@ -45,7 +45,6 @@ def parse():
     ap.add_argument("--workload", default="v0.2-640x368")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     return ap.parse_args()
 
 
@@ -148,6 +147,13 @@ def flop_counts(w, valids):
             "per_euler_step": L * (attn + gemm)}
 
 
+def gemm_flops_per_layer(w, n_sessions):
+    """2 M K N of each projection of one layer (M = sessions x unit tokens)."""
+    m, d, hd, f = n_sessions * w.n_tokens, w.d_model, w.hd, w.d_mlp
+    return {"gemm_qkv": 2 * m * d * 3 * hd, "gemm_o": 2 * m * hd * d,
+            "gemm_up": 2 * m * d * f, "gemm_down": 2 * m * f * d}
+
+
 def append_bytes(w):
     return 2 * 2 * w.n_layers * w.unit_kv_tokens * w.hd * 2   # K and V, read + write, bf16
 
@@ -183,10 +189,17 @@ def traffic_for(kernel_src, table=None):
 # ---------------------------------------------------------------------------
 # CPU baseline: the fp64 oracle on a bounded sample of the same workload
 # ---------------------------------------------------------------------------
-def cpu_sample(w, budget_s):
+# layers of f_theta the CPU baseline times (both arms): each runs over the full cache
+CPU_SAMPLE_LAYERS = 1
+# datasheet figures of a B200, for context next to the measured denominators
+DATASHEET = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+
+def cpu_sample(w, n_layers=CPU_SAMPLE_LAYERS):
     """Time the oracle's f_theta at the bench shapes on a bounded sample: the
-    embedding, as many of the 28 layers as fit the budget (each over the full
-    57,600-token cache), and the head; extrapolate to one Euler step."""
+    embedding, n_layers of the 28 layers (each over the full 57,600-token cache),
+    and the head; extrapolate to one Euler step.  Returns (seconds per Euler step,
+    description): the sample is extrapolated, never a full step."""
     import numpy as np
     import torch
     from threadpoolctl import threadpool_info
@@ -208,34 +221,42 @@ def cpu_sample(w, budget_s):
     t_embed = time.perf_counter() - t0
     pos = valid + np.arange(w.n_tokens)
     layer_times = []
-    t_start = time.perf_counter()
-    while not layer_times or (time.perf_counter() - t_start < budget_s and len(layer_times) < w.n_layers):
+    for _ in range(n_layers):
         t0 = time.perf_counter()
         x = O.layer_forward(cfg, x, lw, kc, vc, pos)
         layer_times.append(time.perf_counter() - t0)
     t0 = time.perf_counter()
     O.head(cfg, x, weights)
     t_head = time.perf_counter() - t0
+    measured = t_embed + sum(layer_times) + t_head
     t_step = t_embed + w.n_layers * statistics.mean(layer_times) + t_head
     threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    sample = (f"oracle f_theta (numpy fp64) at the {w.name} unit over the full {valid}-token cache: "
-              f"embed + {len(layer_times)} of {w.n_layers} layers + head timed, "
-              f"x{w.n_layers}/{len(layer_times)} layers extrapolated to one Euler step")
+    info = {"cores": os.cpu_count(), "threads": threads, "timed_layers": len(layer_times),
+            "extrapolated": True, "measured_s": measured,
+            "sample": (f"oracle f_theta (numpy fp64) at the {w.name} unit over the full "
+                       f"{valid}-token cache: embed + {len(layer_times)} of {w.n_layers} layers "
+                       f"+ head timed, x{w.n_layers}/{len(layer_times)} layers extrapolated to "
+                       "one Euler step")}
     del torch
-    return t_step, threads, sample
+    return t_step, info
 
 
 def run_reference(args, w):
+    """The oracle as the reference arm: each of the K steps times one bounded sample
+    (embedding + CPU_SAMPLE_LAYERS layers over the full cache + head) and extrapolates
+    it to one Euler step; ms_per_step is that extrapolation x the unit's Euler steps,
+    and measured_wall_s the wall time the timed samples actually took."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    budget = max(1.0, min(args.cpu_budget_s, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_sample(w, budget)
+        cpu_sample(w)
     times = []
+    wall0 = time.perf_counter()
     for _ in range(args.steps):
-        t, threads, sample = cpu_sample(w, budget)
+        t, info = cpu_sample(w)
         times.append(t)
+    wall = time.perf_counter() - wall0
     t_step = statistics.mean(times)
     value = 1.0 / t_step
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
@@ -243,8 +264,12 @@ def run_reference(args, w):
             "ms_per_step": t_step * 1e3 * w.n_steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
             "config": config_of(w),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": sample},
+            "extrapolated": True, "timed_layers": info["timed_layers"],
+            "measured_wall_s": wall,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"],
+                             "threads": info["threads"], "kind": "oracle",
+                             "timed_layers": info["timed_layers"], "extrapolated": True,
+                             "sample": info["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -439,6 +464,16 @@ def run_ours(args, w):
         gemm_ms = sum(prof[k][0] for k in ("gemm_qkv", "gemm_o", "gemm_up", "gemm_down"))
         contraction_ms = a_ms + prof["attention_merge"][0] + gemm_ms
         contraction_flop = args.steps * w.n_steps * fl["per_euler_step"]
+        contr_tflops = contraction_flop / (contraction_ms / 1e3) / 1e12
+        # each projection against the measured peaks (2 M K N per launch, L launches per step)
+        gemm_fracs = {}
+        for key, flop in gemm_flops_per_layer(w, len(caps)).items():
+            ms_k = prof[key][0]
+            if ms_k > 0:
+                tf = args.steps * w.n_steps * w.n_layers * flop / (ms_k / 1e3) / 1e12
+                gemm_fracs[key] = {"tflops": tf, "frac": tf / pk["bf16_sustained"],
+                                   "frac_of_burst": tf / pk["bf16"],
+                                   "ms_per_unit": ms_k / args.steps}
         ap_ms, ap_n = prof["append"]
         append_gbs = append_bytes(w) / (ap_ms / max(ap_n, 1) / 1e3) / 1e9 if ap_n else None
         unit_ms = ms_max / args.steps
@@ -457,26 +492,37 @@ def run_ours(args, w):
             "roofline": {"kernel": "attn_tc_kernel (tcgen05 flash attention, split-KV)", "bound": "tensor",
                          "achieved": attn_tflops, "peak": pk["bf16_sustained"],
                          "unit": "TFLOP/s", "frac": attn_tflops / pk["bf16_sustained"],
+                         "frac_of_burst": attn_tflops / pk["bf16"],
+                         "frac_of_datasheet": attn_tflops / DATASHEET["bf16_tflops"],
                          "traffic": traffic,
                          "peak_note": f"{pk['source']} sustained bf16 (kernel timed inside a long step)",
                          "flop_per_launch": fl["attention_per_launch"],
                          "avg_launch_ms": attn_avg_ms,
                          "timing": "CUDA events around each launch on its stream, over a second "
                                    "timed pass of the same steps (direct launches)"},
-            "contractions": {"tflops": contraction_flop / (contraction_ms / 1e3) / 1e12,
-                             "frac_of_bf16_peak": contraction_flop / (contraction_ms / 1e3) / 1e12
-                             / pk["bf16_sustained"],
+            "contractions": {"tflops": contr_tflops,
+                             "frac_of_bf16_peak": contr_tflops / pk["bf16_sustained"],
+                             "frac_of_burst": contr_tflops / pk["bf16"],
+                             "frac_of_datasheet": contr_tflops / DATASHEET["bf16_tflops"],
+                             "projections": gemm_fracs,
                              "attn_gemm_device_ms_per_unit": contraction_ms / args.steps},
             "append": {"gb_s": append_gbs, "frac_of_hbm": (append_gbs / pk["hbm_gbs"]) if append_gbs else None,
+                       "frac_of_datasheet": (append_gbs / DATASHEET["hbm_gbs"]) if append_gbs else None,
                        "bytes": append_bytes(w)},
+            "peaks": {"bf16_sustained_tflops": pk["bf16_sustained"], "bf16_burst_tflops": pk["bf16"],
+                      "hbm_gbs": pk["hbm_gbs"], "source": pk["source"],
+                      "datasheet_bf16_tflops": DATASHEET["bf16_tflops"],
+                      "datasheet_hbm_gbs": DATASHEET["hbm_gbs"]},
             "kernel_ms_per_unit": {k2: round(v2[0] / args.steps, 4) for k2, v2 in prof.items()},
             "profiled_pass_ms_per_step": prof_ms_max / args.steps,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline and n_sess == 1:
-            t_step, threads, sample = cpu_sample(w, args.cpu_budget_s)
-            line["cpu_baseline"] = {"value": 1.0 / t_step, "unit": UNIT, "cores": threads,
-                                    "kind": "oracle", "sample": sample}
+            t_step, info = cpu_sample(w)
+            line["cpu_baseline"] = {"value": 1.0 / t_step, "unit": UNIT, "cores": info["cores"],
+                                    "threads": info["threads"], "kind": "oracle",
+                                    "timed_layers": info["timed_layers"], "extrapolated": True,
+                                    "measured_s": info["measured_s"], "sample": info["sample"]}
         print(json.dumps(line), flush=True)
     p.close()
     if world > 1:

@@ -53,6 +53,9 @@ extern "C" {
 #define SFM_ECUDA         (-4)   /* a CUDA call failed (see sfm_last_cuda_error)  */
 #define SFM_ENOMEM        (-5)   /* device allocation failed in sfm_create        */
 #define SFM_EUNSUPPORTED  (-6)   /* shape the kernels do not support              */
+#define SFM_EDEVICE       (-7)   /* an earlier kernel of this handle gave up a
+                                    bounded wait (see sfm_check_device_error);
+                                    refused until sfm_clear_device_error        */
 
 /* ---- storage / arithmetic type of weights, cache and activations -------- */
 #define SFM_DTYPE_BF16 0   /* bf16 storage, tensor-core MMA with fp32 accumulation;
@@ -145,14 +148,31 @@ SFM_API int sfm_session_get_info(const sfm_handle* h, int session, sfm_session_i
 
 /*
  * Writes the thinker's K/V slice for n_tok / T_u whole units into the
- * session's cache: unit u (u = units_appended + i) goes to slot u mod
- * cache_units, rows verbatim.  k, v: device, [L][n_tok][H][D_h] of the
+ * session's cache ("Wan-Streamer v0.2" digest, "method overview and
+ * architecture", performer path: each rank writes the broadcast, performer-
+ * compatible K/V slice into its pre-allocated local cache; "Wan-Streamer v0.2"
+ * blog, "Infra").  The pages state no eviction policy; here unit u
+ * (u = units_appended + i) goes to slot u mod cache_units, rows verbatim.  k, v: device, [L][n_tok][H][D_h] of the
  * handle's dtype, caller-owned; K is already rotated (post-RoPE).
  * SFM_EINVAL if n_tok is not a positive multiple of T_u; SFM_ECAPACITY if
  * ring == 0 and the units do not fit (nothing is written).
  */
 SFM_API int sfm_kvcache_append(sfm_handle* h, int session, const void* k, const void* v,
                        int n_tok, void* stream);
+
+/*
+ * sfm_kvcache_append for one rank of a head-sharded cache: the broadcast
+ * slice's rows hold src_heads heads ([L][n_tok][src_heads][D_h]) and this
+ * handle's cache keeps heads [head0, head0 + n_heads) of each, n_heads being
+ * the handle's own head count ("Wan-Streamer v0.2" digest, "method overview
+ * and architecture": each performer rank keeps a pre-sharded local cache and
+ * writes the broadcast K/V slice into it; with Ulysses context parallelism a
+ * rank attends over its own head group).  src_heads = n_heads, head0 = 0 is
+ * sfm_kvcache_append.  SFM_EINVAL if the head range does not fit src_heads;
+ * errors and ring behaviour otherwise as for sfm_kvcache_append.
+ */
+SFM_API int sfm_kvcache_append_heads(sfm_handle* h, int session, const void* k, const void* v,
+                                     int n_tok, int src_heads, int head0, void* stream);
 
 /* Copies cache rows [row0, row0 + n_rows) of one layer into caller device
  * buffers k_dst, v_dst ([n_rows][H][D_h]).  Rows index the session's region
@@ -162,7 +182,9 @@ SFM_API int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long l
 
 /*
  * One Euler step of the current unit: v = f_theta(z, tau_from | cache),
- * z <- z + (tau_to - tau_from) v.  z: device fp32 [N][C], N = n_video +
+ * z <- z + (tau_to - tau_from) v ("Wan-Streamer" v0.1 blog, §3.4 conditional
+ * flow matching: the rectified-flow path and its velocity; §3.3: f_theta is the
+ * block-causal Transformer, the unit seeing every cached unit and itself).  z: device fp32 [N][C], N = n_video +
  * n_audio (video rows first), updated in place.  v_out: nullable device fp32
  * [N][C] receiving v, a buffer other than z (SFM_EINVAL otherwise).  The
  * current unit's tokens are at positions p0 + j.
@@ -171,7 +193,11 @@ SFM_API int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_fro
                      float tau_to, float* v_out, void* stream);
 
 /*
- * The whole solve: Euler steps over taus[0] -> taus[1] -> ... -> taus[n-1].
+ * The whole solve: Euler steps over taus[0] -> taus[1] -> ... -> taus[n-1]
+ * (the performer's flow-matching solver for the next unit's audio and video
+ * latents: "Wan-Streamer v0.2" digest, "method overview and architecture";
+ * "Wan-Streamer" v0.1 blog, §3.4 and §5.1).  The pages give neither the step
+ * count nor the schedule; the caller passes the schedule.
  * taus: host array, n_taus >= 2, taus[0] = 1 (z holds eps) decreasing to
  * taus[n-1] = 0 (z then holds the unit's clean latent).  The cache is not
  * modified (the current unit's K/V are scratch, never committed).
@@ -222,6 +248,31 @@ SFM_API int sfm_fm_solve_guided_batched(sfm_handle* h, int n_pairs, const int* s
                                         const int* uncond_sessions, float* const* z,
                                         const float* taus, int n_taus, float scale,
                                         float* const* v_out, void* stream);
+
+/*
+ * Velocities of several consecutive units in one pass of f_theta under the
+ * general block-causal mask ("Wan-Streamer" v0.1 blog, §3.3: a unit sees
+ * itself bidirectionally and every earlier unit, never a later one), the pass a
+ * multi-unit prefill needs (the v0.2 blog's project-page note: a scene goes live
+ * about 0.5 s after its prompt, thinker and performer prefill included).
+ *   - The n_units units follow the session's cache on the timeline: token j of
+ *     unit u is at position p0 + u N + j and sees every valid cached token,
+ *     every token of units <= u and no token of a later unit.  One unit gives
+ *     sfm_denoise_step's velocity.
+ *   - z: host array of n_units device fp32 [N][C] latents (read only), unit u
+ *     at flow time taus[u] (host array).  v_out: host array of n_units distinct
+ *     device fp32 [N][C] buffers (none of them a z) receiving the velocities.
+ *   - commit = 1 appends the units' own K/V, as computed in this pass (at their
+ *     flow times; clean units have tau = 0), to the session's cache as n_units
+ *     units.  Needs unit_kv_tokens == N (SFM_EUNSUPPORTED) and n_units free
+ *     slots (the ring does not wrap here: SFM_ECAPACITY).  commit = 0 changes
+ *     no cache state: the pass's K/V are scratch rows.
+ *   - SFM_ECAPACITY if n_units > max_sessions (activation scratch) or if the
+ *     pass's rows do not fit the session's region: valid_tokens + n_units N <=
+ *     cache_units T_u + N.
+ */
+SFM_API int sfm_velocity_units(sfm_handle* h, int session, int n_units, const float* const* z,
+                               const float* taus, float* const* v_out, int commit, void* stream);
 
 /*
  * Launch mode of sfm_denoise_step / sfm_fm_solve / sfm_fm_solve_batched.
@@ -284,8 +335,11 @@ SFM_API int sfm_attention_block_causal(const void* q, const void* k, const void*
  *   - Returns SFM_ECAPACITY, launching nothing, when the shape needs more
  *     scratch than that (sfm_attention_workspace_bytes(...) is the need).
  *   - The first call on each device resolves the array's device address with
- *     that device current (cudaGetSymbolAddress); make that first call before
- *     any stream capture.
+ *     that device current (cudaGetSymbolAddress) and keeps it for that
+ *     device's context (after a cudaDeviceReset the next call resolves it
+ *     again); make that first call before any stream capture.
+ *   - A bounded wait that gives up inside the kernel is reported through
+ *     sfm_check_call_error, as for the other standalone calls.
  *   - Every call shares the one array per device, and it keeps the last call's
  *     contents (nothing in it needs to start at zero).  Calls that overlap on
  *     the GPU -- on different streams or from different threads -- race on it:
@@ -354,11 +408,63 @@ SFM_API int sfm_profile_end(double* ms, long long* launches);
 SFM_API unsigned long long sfm_kernel_launch_count(void);
 
 /* ---- errors --------------------------------------------------------------- */
-/* Synchronises the device and reads the handle's device error word: 0 when no
- * kernel of this handle has reported a problem; 1 when a bounded wait inside a
- * tensor-core kernel timed out (the kernel then unwound without finishing its
- * tile, so results of that call are invalid). */
+/*
+ * Bounded waits.  Every wait inside the tensor-core kernels (on a TMA load, an
+ * MMA, or another role of the CTA) gives up after a bound (1 s): the waiting
+ * role records its wait site in an error word, the CTA's roles unwind (drain
+ * their own asynchronous copies with bounded waits, free tensor memory, write
+ * zeros for the rows they own) and the kernel returns, so the CUDA context
+ * stays usable.  Results of a call in which a wait gave up are invalid.
+ *
+ * Handle calls.  sfm_check_device_error synchronises the device and returns
+ * the handle's word in *code: 0 when no kernel of the handle gave up, else the
+ * site (0x1nn: a projection kernel, 0x2nn: the attention kernel; nn names the
+ * wait).  Each solve also copies the word to host memory when it ends, so once
+ * that copy has executed, every f_theta call on the handle (sfm_denoise_step,
+ * sfm_fm_solve*, sfm_velocity_units) returns SFM_EDEVICE without launching,
+ * until sfm_clear_device_error (which synchronises the device and zeroes both).
+ *
+ * Standalone calls (sfm_attention*, sfm_linear) share one word per device:
+ * sfm_check_call_error synchronises the current device, returns that word in
+ * *code and zeroes it.
+ */
 SFM_API int sfm_check_device_error(const sfm_handle* h, int* code);
+SFM_API int sfm_clear_device_error(sfm_handle* h);
+SFM_API int sfm_check_call_error(int* code);
+
+/*
+ * Test-only fault injection for the bounded waits (no counterpart in the
+ * method: it exercises the failure path without faulting the GPU).  From the
+ * next launch on, the kernels of handle h (h == NULL: the standalone calls of
+ * this process) run with the given fault bits and wait bound:
+ *   SFM_FAULT_ATTN_NO_LOADS  the attention kernel's TMA producer issues no loads,
+ *   SFM_FAULT_GEMM_NO_LOADS  the projection kernels' TMA producers issue none,
+ * so the roles that wait for those loads give up after wait_ns nanoseconds and
+ * the kernel unwinds.  wait_ns = 0 restores the 1 s bound; otherwise 1e4 <=
+ * wait_ns <= 1e10 (SFM_EINVAL outside, or for unknown fault bits).  faults = 0
+ * and wait_ns = 0 restore normal operation.
+ */
+#define SFM_FAULT_NONE           0
+#define SFM_FAULT_ATTN_NO_LOADS  1
+#define SFM_FAULT_GEMM_NO_LOADS  2
+SFM_API int sfm_test_fault(sfm_handle* h, int faults, long long wait_ns);
+
+/*
+ * The launch plan a handle fixed at create for its four projections (index 0
+ * QKV, 1 O, 2 MLP-up, 3 MLP-down), chosen for a full batch of max_sessions
+ * units: N-tile width, whether the projection runs on CTA pairs
+ * (tcgen05 cta_group::2, 256-row tiles), and its K slices (1 = none).
+ * fused_norm = 1 when every RMSNorm is split between the kernel that updates
+ * the residual (it writes bf16(x g) and partial sums of squares) and the next
+ * projection (bf16 handles).  No counterpart in the method: introspection.
+ */
+typedef struct sfm_plan {
+  int block_n[4];
+  int pair[4];
+  int k_splits[4];
+  int fused_norm;
+} sfm_plan;
+SFM_API int sfm_get_plan(const sfm_handle* h, sfm_plan* out);
 SFM_API const char* sfm_strerror(int status);
 /* The cudaError_t of the last failed CUDA call made by this library on this
  * host thread (0 if none). */

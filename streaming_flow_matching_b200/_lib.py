@@ -13,6 +13,8 @@ LIB_PATH = os.path.join(_HERE, "libsfm.so")
 
 SFM_OK, SFM_EINVAL, SFM_ECAPACITY, SFM_ESESSION, SFM_ECUDA, SFM_ENOMEM, SFM_EUNSUPPORTED = (
     0, -1, -2, -3, -4, -5, -6)
+SFM_EDEVICE = -7
+SFM_FAULT_NONE, SFM_FAULT_ATTN_NO_LOADS, SFM_FAULT_GEMM_NO_LOADS = 0, 1, 2
 SFM_DTYPE_BF16, SFM_DTYPE_FP32 = 0, 1
 SFM_NOALLOC_SCRATCH_BYTES = 64 << 20
 SFM_LINEAR_F32, SFM_LINEAR_OUT, SFM_LINEAR_GELU, SFM_LINEAR_RESID = 0, 1, 2, 3
@@ -40,6 +42,11 @@ class sfm_session_info(C.Structure):
                 ("valid_tokens", C.c_longlong), ("p0", C.c_longlong), ("base_row", C.c_longlong)]
 
 
+class sfm_plan(C.Structure):
+    _fields_ = [("block_n", C.c_int * 4), ("pair", C.c_int * 4), ("k_splits", C.c_int * 4),
+                ("fused_norm", C.c_int)]
+
+
 class SfmError(RuntimeError):
     def __init__(self, status, what=""):
         self.status = status
@@ -63,6 +70,7 @@ def _load():
         "sfm_session_reset": (i, [vp, i]),
         "sfm_session_get_info": (i, [vp, i, C.POINTER(sfm_session_info)]),
         "sfm_kvcache_append": (i, [vp, i, vp, vp, i, vp]),
+        "sfm_kvcache_append_heads": (i, [vp, i, vp, vp, i, i, i, vp]),
         "sfm_kvcache_read": (i, [vp, i, i, ll, ll, vp, vp, vp]),
         "sfm_denoise_step": (i, [vp, i, vp, f, f, vp, vp]),
         "sfm_fm_solve": (i, [vp, i, vp, C.POINTER(f), i, vp]),
@@ -70,6 +78,7 @@ def _load():
         "sfm_fm_solve_guided": (i, [vp, i, i, vp, C.POINTER(f), i, f, vp]),
         "sfm_fm_solve_guided_batched": (i, [vp, i, C.POINTER(i), C.POINTER(i), C.POINTER(vp),
                                             C.POINTER(f), i, f, C.POINTER(vp), vp]),
+        "sfm_velocity_units": (i, [vp, i, i, C.POINTER(vp), C.POINTER(f), C.POINTER(vp), i, vp]),
         "sfm_set_graph_mode": (i, [vp, i]),
         "sfm_attention_workspace_bytes": (sz, [i, i, i, i, i]),
         "sfm_attention": (i, [vp, vp, vp, vp, i, i, i, i, i, vp, sz, vp]),
@@ -77,6 +86,10 @@ def _load():
         "sfm_attention_noalloc": (i, [vp, vp, vp, vp, i, i, i, i, i, vp]),
         "sfm_linear": (i, [vp, vp, vp, i, i, i, i, i, vp]),
         "sfm_check_device_error": (i, [vp, C.POINTER(i)]),
+        "sfm_clear_device_error": (i, [vp]),
+        "sfm_check_call_error": (i, [C.POINTER(i)]),
+        "sfm_test_fault": (i, [vp, i, ll]),
+        "sfm_get_plan": (i, [vp, C.POINTER(sfm_plan)]),
         "sfm_euler_update": (i, [vp, vp, f, ll, vp]),
         "sfm_fm_solve_exact_velocity": (i, [vp, vp, vp, C.POINTER(f), i, vp]),
         "sfm_profile_begin": (i, [i]),
@@ -97,12 +110,15 @@ lib = _load()
 
 # Every symbol declared in include/sfm.h, in declaration order.
 EXPORTS = ["sfm_create", "sfm_destroy", "sfm_session_open", "sfm_session_reset",
-           "sfm_session_get_info", "sfm_kvcache_append", "sfm_kvcache_read", "sfm_denoise_step",
+           "sfm_session_get_info", "sfm_kvcache_append", "sfm_kvcache_append_heads",
+           "sfm_kvcache_read", "sfm_denoise_step",
            "sfm_fm_solve", "sfm_fm_solve_batched", "sfm_fm_solve_guided",
-           "sfm_fm_solve_guided_batched", "sfm_set_graph_mode", "sfm_attention_workspace_bytes",
-           "sfm_attention", "sfm_attention_block_causal", "sfm_attention_noalloc", "sfm_linear", "sfm_euler_update", "sfm_fm_solve_exact_velocity", "sfm_profile_begin", "sfm_profile_end",
-           "sfm_kernel_launch_count", "sfm_check_device_error", "sfm_strerror",
-           "sfm_last_cuda_error"]
+           "sfm_fm_solve_guided_batched", "sfm_velocity_units", "sfm_set_graph_mode",
+           "sfm_attention_workspace_bytes", "sfm_attention", "sfm_attention_block_causal",
+           "sfm_attention_noalloc", "sfm_linear", "sfm_euler_update", "sfm_fm_solve_exact_velocity",
+           "sfm_profile_begin", "sfm_profile_end", "sfm_kernel_launch_count",
+           "sfm_check_device_error", "sfm_clear_device_error", "sfm_check_call_error",
+           "sfm_test_fault", "sfm_get_plan", "sfm_strerror", "sfm_last_cuda_error"]
 
 PROF_KINDS = ["append", "attention", "attention_merge", "gemm_qkv", "gemm_o", "gemm_up",
               "gemm_down", "rowops", "head_euler"]
@@ -118,6 +134,18 @@ def profile_end():
     n = (C.c_longlong * len(PROF_KINDS))()
     check(lib.sfm_profile_end(ms, n), "sfm_profile_end")
     return {k: (ms[i], n[i]) for i, k in enumerate(PROF_KINDS)}
+
+
+def check_call_error():
+    """Synchronises the current device; returns and clears the standalone calls' error word."""
+    code = C.c_int()
+    check(lib.sfm_check_call_error(C.byref(code)), "sfm_check_call_error")
+    return code.value
+
+
+def set_call_fault(faults, wait_ns=0):
+    """Test-only: fault bits and wait bound of the standalone calls (0, 0 = normal)."""
+    check(lib.sfm_test_fault(None, faults, wait_ns), "sfm_test_fault")
 
 
 def check(status, what=""):

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 
 #include "attn.cuh"
@@ -12,6 +13,12 @@
 #include "sm100.cuh"
 
 using namespace sfm;
+
+namespace {
+// Error word of the standalone calls (sfm_attention*, sfm_linear): one per device
+// that loads the library, like every file-scope device variable.
+__device__ int g_call_err;
+}  // namespace
 
 namespace sfm {
 static thread_local int g_last_cuda_error = 0;
@@ -37,7 +44,7 @@ struct sfm_handle {
   // solves run as one CUDA graph, captured on a private stream and updated in place
   bool graphs = true;
   cudaStream_t cap_stream = nullptr;
-  cudaGraphExec_t graph_exec[2] = {nullptr, nullptr};   // plain / guided solves
+  cudaGraphExec_t graph_exec[3] = {nullptr, nullptr, nullptr};   // plain / guided / units passes
   long long pool_used = 0;
   std::vector<Session> sessions;
   // scratch, sized for max_sessions * n_tok rows
@@ -53,6 +60,8 @@ struct sfm_handle {
   float* o_part = nullptr;   // [kMaxSplits][M][H][D]
   float* lse_part = nullptr; // [kMaxSplits][M][H]
   int* d_err = nullptr;      // device error word (bounded waits that timed out)
+  volatile int* h_err = nullptr;   // pinned host copy of d_err, written at the end of each solve
+  Guard gd;                  // d_err, wait bound and test-only faults of this handle's kernels
   int sms = 148;
   // TMA tensor maps (bf16 mode): activations over max_sessions * N rows, weights per layer
   CUtensorMap map_xn{}, map_ao{}, map_hmlp{};
@@ -167,7 +176,7 @@ int make_rows_map(CUtensorMap* m, const void* p, long long rows, int heads, int 
   return make_tmap_bf16(m, p, 3, dims, strides, box);
 }
 
-GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err, int block_n,
+GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, const Guard& gd, int block_n,
                    bool pair) {
   GemmArgs g{};
   g.M = M;
@@ -176,7 +185,9 @@ GemmArgs gemm_args(int M, int N, int K, int epi, void* C, int ldc, int* err, int
   g.epi = epi;
   g.C = C;
   g.ldc = ldc;
-  g.err = err;
+  g.err = gd.err;
+  g.wait_ns = gd.wait_ns;
+  g.fault = gd.fault;
   g.hd = 0;
   g.block_n = block_n;
   g.pair = pair ? 1 : 0;
@@ -190,8 +201,9 @@ struct Guidance {
 
 // One Euler step of f_theta for the sessions in b (RoPE table already filled).
 // Guided: entries 2p, 2p + 1 are a conditional / unconditional pair sharing z[2p].
-int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from, float tau_to,
-             float* const* v_out, const Guidance& gd, cudaStream_t s) {
+int run_step(sfm_handle* h, const BatchDesc& b, const AttnDesc& ad, float* const* z,
+             float tau_from, float tau_to, float* const* v_out, const Guidance& gd,
+             cudaStream_t s) {
   const sfm_config& c = h->cfg;
   const int M = b.n * b.n_tok;
   const int d = c.d_model, hd = h->hd, F = c.d_mlp, dt = c.dtype;
@@ -227,7 +239,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
   // next norm's numerator and the row's whole sum of squares)
   auto resid_split = [&](const CUtensorMap& ma, const CUtensorMap& mb, int K, int bn, int slices,
                          const void* gain) {
-    GemmArgs g = gemm_args(M, d, K, EPI_F32, h->ws_splitk, d, h->d_err, bn, false);
+    GemmArgs g = gemm_args(M, d, K, EPI_F32, h->ws_splitk, d, h->gd, bn, false);
     g.k_splits = slices;
     int r = launch_gemm_tc(ma, mb, g, h->sms, s);
     if (!r)
@@ -244,7 +256,6 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
     ss_n = d / bn;
     return g;
   };
-  const AttnDesc ad = attn_desc(b);
   const int splits = tc ? attention_tc_splits_batch(ad, c.n_heads, h->sms) : 1;
   for (int l = 0; l < c.n_layers; ++l) {
     if (!tc) {
@@ -255,7 +266,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       // QKV projection with the norm's 1 / rms, RoPE and the cache-tail scatter fused in
       // the epilogue
       ProfScope ps(SFM_PROF_GEMM_QKV, s);
-      GemmArgs g = normed(gemm_args(M, 3 * hd, d, EPI_QKV, nullptr, 0, h->d_err, h->bn_qkv, h->pair_qkv));
+      GemmArgs g = normed(gemm_args(M, 3 * hd, d, EPI_QKV, nullptr, 0, h->gd, h->bn_qkv, h->pair_qkv));
       g.cos_t = h->cos_t;
       g.sin_t = h->sin_t;
       g.q_out = (__nv_bfloat16*)h->q;
@@ -276,7 +287,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
     if (tc) {
       SFM_TRY(launch_attention_tc(h->map_q, h->map_kpool, h->map_vpool, ad,
                                   (int)((long long)l * c.pool_tokens), c.n_heads, splits, h->ao,
-                                  h->o_part, h->lse_part, h->d_err, s));
+                                  h->o_part, h->lse_part, h->gd, s));
     } else {
       SFM_TRY(launch_attention(ad, h->q, h->layer_k(l), h->layer_v(l), h->ao, c.n_heads,
                                c.head_dim, dt, splits, h->o_part, h->lse_part, s));
@@ -287,7 +298,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
         SFM_TRY(resid_split(h->map_ao, h->map_wo[l], hd, h->bn_o, h->ksplit_o, h->g_mlp[l]));
       } else if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_ao, h->map_wo[l],
-                               norm_next(gemm_args(M, d, hd, EPI_RESID, h->x, d, h->d_err, h->bn_o, h->pair_o),
+                               norm_next(gemm_args(M, d, hd, EPI_RESID, h->x, d, h->gd, h->bn_o, h->pair_o),
                                          h->g_mlp[l], h->bn_o),
                                h->sms, s));
       } else {
@@ -302,7 +313,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
       ProfScope ps(SFM_PROF_GEMM_UP, s);
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_xn, h->map_w1[l],
-                               normed(gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->d_err, h->bn_up, h->pair_up)),
+                               normed(gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->gd, h->bn_up, h->pair_up)),
                                h->sms, s));
       } else {
         SFM_TRY(launch_gemm(h->xn, h->w_1[l], h->hmlp, M, F, d, EPI_GELU, dt, s));
@@ -315,7 +326,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
                             l + 1 < c.n_layers ? h->g_attn[l + 1] : nullptr));
       } else if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_hmlp, h->map_w2[l],
-                               norm_next(gemm_args(M, d, F, EPI_RESID, h->x, d, h->d_err, h->bn_down, h->pair_down),
+                               norm_next(gemm_args(M, d, F, EPI_RESID, h->x, d, h->gd, h->bn_down, h->pair_down),
                                          l + 1 < c.n_layers ? h->g_attn[l + 1] : nullptr, h->bn_down),
                                h->sms, s));
       } else {
@@ -332,6 +343,22 @@ int run_step(sfm_handle* h, const BatchDesc& b, float* const* z, float tau_from,
   return SFM_OK;
 }
 
+// The device error word goes to pinned host memory at the end of every solve, so
+// a later call can refuse (SFM_EDEVICE) without synchronising.
+int error_to_host(sfm_handle* h, cudaStream_t s) {
+  if (!h->h_err) return SFM_OK;
+  const cudaError_t e =
+      cudaMemcpyAsync((void*)h->h_err, h->d_err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) return SFM_OK;
+  g_last_cuda_error = (int)e;
+  return SFM_ECUDA;
+}
+
+// SFM_EDEVICE once a solve's copy of the error word has reported a timed-out wait.
+int device_error_pending(const sfm_handle* h) {
+  return h->h_err && *h->h_err ? SFM_EDEVICE : SFM_OK;
+}
+
 int check_taus(const float* taus, int n_taus) {
   if (!taus || n_taus < 2) return SFM_EINVAL;
   for (int i = 0; i < n_taus; ++i)
@@ -339,21 +366,27 @@ int check_taus(const float* taus, int n_taus) {
   return SFM_OK;
 }
 
-int solve_direct(sfm_handle* h, int n, const int* sessions, float* const* z, const float* taus,
-                 int n_taus, float* const* v_out, const Guidance& gd, cudaStream_t s) {
+// The batch of one pass of f_theta and the attention over it: the sessions of a
+// (batched, guided) solve, each seeing its whole cache and unit; or several units
+// of one session under the general block-causal mask.
+struct Pass {
   BatchDesc b;
-  fill_batch(h, n, sessions, &b);
+  AttnDesc a;
+};
+
+int solve_direct(sfm_handle* h, const Pass& ps, float* const* z, const float* taus, int n_taus,
+                 float* const* v_out, const Guidance& gd, cudaStream_t s) {
   int rc;
   {
-    ProfScope ps(SFM_PROF_ROWOPS, s);
-    rc = launch_rope_table(b, h->cos_t, h->sin_t, h->cfg.head_dim, h->cfg.rope_theta, s);
+    ProfScope prof(SFM_PROF_ROWOPS, s);
+    rc = launch_rope_table(ps.b, h->cos_t, h->sin_t, h->cfg.head_dim, h->cfg.rope_theta, s);
   }
   if (rc) return rc;
   for (int i = 0; i + 1 < n_taus; ++i) {
-    rc = run_step(h, b, z, taus[i], taus[i + 1], v_out, gd, s);
+    rc = run_step(h, ps.b, ps.a, z, taus[i], taus[i + 1], v_out, gd, s);
     if (rc) return rc;
   }
-  return SFM_OK;
+  return error_to_host(h, s);
 }
 
 // A solve is several hundred small launches (8 per layer per Euler step).  They
@@ -363,14 +396,14 @@ int solve_direct(sfm_handle* h, int n, const int* sessions, float* const* z, con
 // cache lengths, latent pointers), so repeated units pay neither instantiation
 // nor per-launch overheads.  The profiler brackets every launch with events,
 // so a profiled call launches directly.
-int solve(sfm_handle* h, int n, const int* sessions, float* const* z, const float* taus,
-          int n_taus, float* const* v_out, cudaStream_t s, const Guidance& gd = Guidance{}) {
+int solve_pass(sfm_handle* h, const Pass& ps, float* const* z, const float* taus, int n_taus,
+               float* const* v_out, cudaStream_t s, const Guidance& gd, int kind) {
   if (!h->graphs || !h->cap_stream || profiling_active())
-    return solve_direct(h, n, sessions, z, taus, n_taus, v_out, gd, s);
-  cudaGraphExec_t& exec = h->graph_exec[gd.on ? 1 : 0];
+    return solve_direct(h, ps, z, taus, n_taus, v_out, gd, s);
+  cudaGraphExec_t& exec = h->graph_exec[kind];
   if (cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess)
     return record_cuda(cudaGetLastError());
-  const int rc = solve_direct(h, n, sessions, z, taus, n_taus, v_out, gd, h->cap_stream);
+  const int rc = solve_direct(h, ps, z, taus, n_taus, v_out, gd, h->cap_stream);
   cudaGraph_t g = nullptr;
   const cudaError_t ec = cudaStreamEndCapture(h->cap_stream, &g);
   if (rc || ec != cudaSuccess || !g) {
@@ -394,6 +427,18 @@ int solve(sfm_handle* h, int n, const int* sessions, float* const* z, const floa
     return record_cuda(e);
   }
   return record_cuda(cudaGraphLaunch(exec, s));
+}
+
+// Graph slots of the three kinds of pass (different kernels, so each keeps its own
+// executable graph and alternating them costs no re-instantiation).
+constexpr int kGraphPlain = 0, kGraphGuided = 1, kGraphUnits = 2;
+
+int solve(sfm_handle* h, int n, const int* sessions, float* const* z, const float* taus,
+          int n_taus, float* const* v_out, cudaStream_t s, const Guidance& gd = Guidance{}) {
+  Pass ps;
+  fill_batch(h, n, sessions, &ps.b);
+  ps.a = attn_desc(ps.b);
+  return solve_pass(h, ps, z, taus, n_taus, v_out, s, gd, gd.on ? kGraphGuided : kGraphPlain);
 }
 
 }  // namespace
@@ -464,6 +509,17 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     }
   }
   if (!rc) rc = dalloc(h, &h->d_err, sizeof(int));
+  if (!rc) {
+    void* hp = nullptr;
+    if (cudaHostAlloc(&hp, sizeof(int), cudaHostAllocDefault) != cudaSuccess) {
+      cudaGetLastError();
+      rc = SFM_ENOMEM;
+    } else {
+      h->h_err = (volatile int*)hp;
+      *h->h_err = 0;
+    }
+    h->gd.err = h->d_err;
+  }
   // Zero everything once: rows a tile reads past a session's valid range must hold
   // finite values, never uninitialised bit patterns.
   if (!rc) {
@@ -546,6 +602,7 @@ void sfm_destroy(sfm_handle* h) {
     if (e) cudaGraphExecDestroy(e);
   if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   for (void* p : h->owned) cudaFree(p);
+  if (h->h_err) cudaFreeHost((void*)h->h_err);
   delete h;
 }
 
@@ -590,11 +647,22 @@ int sfm_session_get_info(const sfm_handle* h, int session, sfm_session_info* out
   return SFM_OK;
 }
 
-int sfm_kvcache_append(sfm_handle* h, int session, const void* k, const void* v, int n_tok,
-                       void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Appends n_tok / T_u units of a slice whose rows hold src_heads heads; the cache
+// takes heads [head0, head0 + H) of each row (all of them when src_heads == H).
+int kvcache_append(sfm_handle* h, int session, const void* k, const void* v, int n_tok,
+                   int src_heads, int head0, void* stream) {
   int rc = session_ok(h, session);
   if (rc) return rc;
   if (!k || !v || !aligned16(k) || !aligned16(v)) return SFM_EINVAL;
+  const int H = h->cfg.n_heads;
+  if (src_heads < H || head0 < 0 || head0 + H > src_heads) return SFM_EINVAL;
+  const int src_row_bytes = src_heads * h->cfg.head_dim * h->es;
+  const int src_off_bytes = head0 * h->cfg.head_dim * h->es;
+  if (src_off_bytes % 16 || src_row_bytes % 16) return SFM_EINVAL;
   const int T = h->cfg.unit_kv_tokens;
   if (n_tok <= 0 || n_tok % T) return SFM_EINVAL;
   Session& s = h->sessions[session];
@@ -604,28 +672,45 @@ int sfm_kvcache_append(sfm_handle* h, int session, const void* k, const void* v,
   long long skip = n_units > s.cache_units ? n_units - s.cache_units : 0;
   const long long first = s.units + skip;
   const size_t row_bytes = (size_t)h->hd * h->es;
-  const char* ks = (const char*)k + skip * T * row_bytes;
-  const char* vs = (const char*)v + skip * T * row_bytes;
+  const char* ks = (const char*)k + skip * T * (size_t)src_row_bytes;
+  const char* vs = (const char*)v + skip * T * (size_t)src_row_bytes;
   // the kernel reads rows layer * n_tok + t of the caller's slice; with a skip,
   // each layer's rows start skip * T rows later inside that layer
   ProfScope ps(SFM_PROF_APPEND, (cudaStream_t)stream);
   if (skip) {
     // copy layer by layer so the per-layer source stride stays n_tok
     for (int l = 0; l < h->cfg.n_layers; ++l) {
-      rc = launch_kv_append(ks + (size_t)l * n_tok * row_bytes, vs + (size_t)l * n_tok * row_bytes,
-                            h->layer_k(l), h->layer_v(l), 1, h->cfg.pool_tokens, (int)row_bytes,
-                            (int)((n_units - skip) * T), T, s.base_row, first % s.cache_units,
-                            s.cache_units, (cudaStream_t)stream);
+      rc = launch_kv_append(ks + (size_t)l * n_tok * src_row_bytes,
+                            vs + (size_t)l * n_tok * src_row_bytes, h->layer_k(l), h->layer_v(l),
+                            1, h->cfg.pool_tokens, (int)row_bytes, (int)((n_units - skip) * T), T,
+                            s.base_row, first % s.cache_units, s.cache_units, (cudaStream_t)stream,
+                            src_row_bytes, src_off_bytes);
       if (rc) return rc;
     }
   } else {
     rc = launch_kv_append(k, v, h->k_pool, h->v_pool, h->cfg.n_layers, h->cfg.pool_tokens,
                           (int)row_bytes, n_tok, T, s.base_row, first % s.cache_units,
-                          s.cache_units, (cudaStream_t)stream);
+                          s.cache_units, (cudaStream_t)stream, src_row_bytes, src_off_bytes);
     if (rc) return rc;
   }
   s.units += n_units;
   return SFM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sfm_kvcache_append(sfm_handle* h, int session, const void* k, const void* v, int n_tok,
+                       void* stream) {
+  if (!h) return SFM_EINVAL;
+  return kvcache_append(h, session, k, v, n_tok, h->cfg.n_heads, 0, stream);
+}
+
+int sfm_kvcache_append_heads(sfm_handle* h, int session, const void* k, const void* v, int n_tok,
+                             int src_heads, int head0, void* stream) {
+  if (!h) return SFM_EINVAL;
+  return kvcache_append(h, session, k, v, n_tok, src_heads, head0, stream);
 }
 
 int sfm_kvcache_read(const sfm_handle* h, int session, int layer, long long row0,
@@ -661,6 +746,7 @@ int sfm_denoise_step(sfm_handle* h, int session, float* z, float tau_from, float
   if (rc) return rc;
   if (!h->has_weights || !z || !isfinite(tau_from) || !isfinite(tau_to)) return SFM_EINVAL;
   if (v_out == z) return SFM_EINVAL;   // the step writes both
+  if ((rc = device_error_pending(h))) return rc;
   const float taus[2] = {tau_from, tau_to};
   float* zs[1] = {z};
   float* vs[1] = {v_out};
@@ -673,6 +759,7 @@ int sfm_fm_solve(sfm_handle* h, int session, float* z, const float* taus, int n_
   if (rc) return rc;
   if (!h->has_weights || !z) return SFM_EINVAL;
   if ((rc = check_taus(taus, n_taus))) return rc;
+  if ((rc = device_error_pending(h))) return rc;
   float* zs[1] = {z};
   return solve(h, 1, &session, zs, taus, n_taus, nullptr, (cudaStream_t)stream);
 }
@@ -692,6 +779,7 @@ int sfm_fm_solve_batched(sfm_handle* h, int n_sessions, const int* sessions, flo
       if (sessions[j] == sessions[i] || z[j] == z[i]) return SFM_EINVAL;
   }
   if ((rc = check_taus(taus, n_taus))) return rc;
+  if ((rc = device_error_pending(h))) return rc;
   return solve(h, n_sessions, sessions, z, taus, n_taus, nullptr, (cudaStream_t)stream);
 }
 
@@ -725,6 +813,7 @@ int sfm_fm_solve_guided_batched(sfm_handle* h, int n_pairs, const int* sessions,
       if (ids[j] == ids[i]) return SFM_EINVAL;
   }
   if ((rc = check_taus(taus, n_taus))) return rc;
+  if ((rc = device_error_pending(h))) return rc;
   Guidance gd;
   gd.on = true;
   gd.scale = scale;
@@ -735,6 +824,59 @@ int sfm_fm_solve_guided(sfm_handle* h, int session, int uncond_session, float* z
                         const float* taus, int n_taus, float scale, void* stream) {
   return sfm_fm_solve_guided_batched(h, 1, &session, &uncond_session, &z, taus, n_taus, scale,
                                      nullptr, stream);
+}
+
+int sfm_velocity_units(sfm_handle* h, int session, int n_units, const float* const* z,
+                       const float* taus, float* const* v_out, int commit, void* stream) {
+  int rc = session_ok(h, session);
+  if (rc) return rc;
+  if (!h->has_weights || !z || !taus || !v_out || n_units < 1 || (commit != 0 && commit != 1))
+    return SFM_EINVAL;
+  if (n_units > h->cfg.max_sessions || n_units > kMaxBatch) return SFM_ECAPACITY;
+  for (int u = 0; u < n_units; ++u) {
+    if (!z[u] || !v_out[u] || !isfinite(taus[u])) return SFM_EINVAL;
+    for (int q = 0; q < n_units; ++q)
+      if (v_out[u] == z[q] || (q < u && v_out[q] == v_out[u])) return SFM_EINVAL;
+  }
+  Session& se = h->sessions[session];
+  const long long N = h->n_tok, T = h->cfg.unit_kv_tokens;
+  const long long valid = valid_tokens(h, se);
+  // the pass's own K/V go to the rows after the valid cache: they must fit the
+  // session's region (its slots plus the unit's scratch rows)
+  if (valid + n_units * N > (long long)se.cache_units * T + N) return SFM_ECAPACITY;
+  if (commit) {
+    if (T != N) return SFM_EUNSUPPORTED;              // a committed unit is one cache unit
+    if (se.units + n_units > se.cache_units) return SFM_ECAPACITY;   // no ring wrap
+  }
+  if ((rc = device_error_pending(h))) return rc;
+  Pass ps;
+  BatchDesc& b = ps.b;
+  memset(&b, 0, sizeof(b));
+  b.n = n_units;
+  b.n_tok = (int)N;
+  b.n_video = h->cfg.n_video;
+  b.per_tau = 1;
+  for (int u = 0; u < n_units; ++u) {
+    b.base[u] = se.base_row;
+    b.valid[u] = (int)(valid + u * N);           // unit u's K/V rows follow the earlier units'
+    b.p0[u] = se.units * T + u * N;
+    b.tau[u] = taus[u];
+  }
+  AttnDesc& a = ps.a;
+  memset(&a, 0, sizeof(a));
+  a.n = 1;
+  a.rows_per = (int)(n_units * N);
+  a.unit_rows = (int)N;
+  a.kbase[0] = se.base_row;
+  a.nkeys[0] = (int)(valid + n_units * N);
+  // one step of zero length: the head kernel writes v and leaves z as it is
+  const float zero_step[2] = {0.f, 0.f};
+  // the latents are only read (a zero-length step writes no z)
+  rc = solve_pass(h, ps, const_cast<float* const*>(z), zero_step, 2, v_out, (cudaStream_t)stream,
+                  Guidance{}, kGraphUnits);
+  if (rc) return rc;
+  if (commit) se.units += n_units;               // the rows are the next slots already
+  return SFM_OK;
 }
 
 // The standalone call chooses its split count for a 148-SM B200 whatever the
@@ -750,6 +892,68 @@ size_t sfm_attention_workspace_bytes(int n_q, int n_kv, int n_heads, int head_di
 }  // extern "C"
 
 namespace {
+
+// Device address of g_call_err in the current context.  The address is kept per
+// (device, context): after a cudaDeviceReset the primary context, and with it the
+// module holding the variable, is new, so the address is resolved again.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+std::mutex g_err_mu;
+CtxGetCurrentFn g_ctx_current = nullptr;
+struct ErrSlot {
+  CUcontext ctx = nullptr;
+  int* ptr = nullptr;
+};
+ErrSlot g_err_slot[64];
+int g_call_fault = 0;
+unsigned long long g_call_wait_ns = 0;
+
+}  // namespace
+
+namespace sfm {
+int current_context(void** ctx) {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = (CtxGetCurrentFn)fn;
+    else
+      cudaGetLastError();
+  });
+  CUcontext c = nullptr;
+  if (!g_ctx_current || g_ctx_current(&c) != CUDA_SUCCESS) return SFM_ECUDA;
+  *ctx = (void*)c;
+  return SFM_OK;
+}
+}  // namespace sfm
+
+namespace {
+
+int call_guard(Guard* gd) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda(e);
+  if (dev < 0 || dev >= 64) return SFM_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  CUcontext ctx = nullptr;
+  if (current_context((void**)&ctx)) return SFM_ECUDA;
+  ErrSlot& slot = g_err_slot[dev];
+  if (!ctx || slot.ctx != ctx || !slot.ptr) {
+    // resolving the symbol also makes the runtime bring up the device's context
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_call_err);
+    if (e != cudaSuccess || !p) return record_cuda(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+    if (!ctx && (current_context((void**)&ctx) || !ctx)) return SFM_ECUDA;
+    slot.ctx = ctx;
+    slot.ptr = (int*)p;
+  }
+  gd->err = slot.ptr;
+  gd->fault = g_call_fault;
+  if (g_call_wait_ns) gd->wait_ns = g_call_wait_ns;
+  return SFM_OK;
+}
 
 // Standalone attention, every key visible (unit_tokens = 0) or block-causal over
 // query units of unit_tokens with the first n_kv - n_q keys a shared prefix.
@@ -788,9 +992,10 @@ int attention_call(const void* q, const void* k, const void* v, void* o, int n_q
   int rc = make_rows_map(&mq, q, n_q, n_heads, kAttnQBoxRows);
   if (!rc) rc = make_rows_map(&mk, k, n_kv, n_heads, kAttnKVBoxRows);
   if (!rc) rc = make_rows_map(&mv, v, n_kv, n_heads, kAttnKVBoxRows);
+  Guard gd;
+  if (!rc) rc = call_guard(&gd);
   if (rc) return rc;
-  return launch_attention_tc(mq, mk, mv, a, 0, n_heads, splits, o, o_part, lse_part, nullptr,
-                             stream);
+  return launch_attention_tc(mq, mk, mv, a, 0, n_heads, splits, o, o_part, lse_part, gd, stream);
 }
 
 }  // namespace
@@ -836,9 +1041,65 @@ int sfm_euler_update(float* z, const float* v, float dtau, long long n, void* st
 int sfm_check_device_error(const sfm_handle* h, int* code) {
   if (!h || !code) return SFM_EINVAL;
   int v = 0;
-  const cudaError_t e = cudaMemcpy(&v, h->d_err, sizeof(int), cudaMemcpyDeviceToHost);
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&v, h->d_err, sizeof(int), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return record_cuda(e);
   *code = v;
+  return SFM_OK;
+}
+
+int sfm_clear_device_error(sfm_handle* h) {
+  if (!h) return SFM_EINVAL;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemset(h->d_err, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return record_cuda(e);
+  if (h->h_err) *h->h_err = 0;
+  return SFM_OK;
+}
+
+int sfm_check_call_error(int* code) {
+  if (!code) return SFM_EINVAL;
+  Guard gd;
+  int rc = call_guard(&gd);
+  if (rc) return rc;
+  int v = 0;
+  const int zero = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&v, gd.err, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(gd.err, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return record_cuda(e);
+  *code = v;
+  return SFM_OK;
+}
+
+int sfm_test_fault(sfm_handle* h, int faults, long long wait_ns) {
+  if (faults & ~(SFM_FAULT_ATTN_NO_LOADS | SFM_FAULT_GEMM_NO_LOADS)) return SFM_EINVAL;
+  if (wait_ns != 0 && (wait_ns < 10000LL || wait_ns > 10000000000LL)) return SFM_EINVAL;
+  const unsigned long long ns = wait_ns ? (unsigned long long)wait_ns : sm100::kWaitNs;
+  if (h) {
+    h->gd.fault = faults;
+    h->gd.wait_ns = ns;
+  } else {
+    std::lock_guard<std::mutex> lock(g_err_mu);
+    g_call_fault = faults;
+    g_call_wait_ns = wait_ns ? ns : 0;
+  }
+  return SFM_OK;
+}
+
+int sfm_get_plan(const sfm_handle* h, sfm_plan* out) {
+  if (!h || !out) return SFM_EINVAL;
+  memset(out, 0, sizeof(*out));
+  const int bn[4] = {h->bn_qkv, h->bn_o, h->bn_up, h->bn_down};
+  const bool pr[4] = {h->pair_qkv, h->pair_o, h->pair_up, h->pair_down};
+  const int ks[4] = {1, h->ksplit_o, 1, h->ksplit_down};
+  for (int i = 0; i < 4; ++i) {
+    out->block_n[i] = bn[i];
+    out->pair[i] = pr[i] ? 1 : 0;
+    out->k_splits[i] = ks[i];
+  }
+  out->fused_norm = h->has_weights && h->cfg.dtype == SFM_DTYPE_BF16 ? 1 : 0;
   return SFM_OK;
 }
 
@@ -869,8 +1130,10 @@ int sfm_linear(const void* x, const void* w, void* y, int M, int N, int K, int e
   CUtensorMap ma, mb;
   int rc = make_a_map(&ma, x, M, K);
   if (!rc) rc = make_b_map(&mb, w, N, K, pair ? bn / 2 : bn);
+  Guard gd;
+  if (!rc) rc = call_guard(&gd);
   if (rc) return rc;
-  return launch_gemm_tc(ma, mb, gemm_args(M, N, K, epi, y, N, nullptr, bn, pair), sms,
+  return launch_gemm_tc(ma, mb, gemm_args(M, N, K, epi, y, N, gd, bn, pair), sms,
                         (cudaStream_t)stream);
 }
 
@@ -883,6 +1146,7 @@ const char* sfm_strerror(int status) {
     case SFM_ECUDA: return "CUDA error";
     case SFM_ENOMEM: return "device allocation failed";
     case SFM_EUNSUPPORTED: return "unsupported shape";
+    case SFM_EDEVICE: return "a kernel gave up a bounded wait (clear with sfm_clear_device_error)";
     default: return "unknown status";
   }
 }

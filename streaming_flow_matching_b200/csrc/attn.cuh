@@ -51,8 +51,9 @@ int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys
 int attention_tc_splits_batch(const AttnDesc& a, int n_heads, int sms);
 // mq: map over the query rows [rows][H][128]; mk, mv: maps over the key rows, of
 // which this call uses rows kv_row0 + kbase[s] + [0, nkeys[s]).
+// gd: error word, wait bound and test-only fault of the launch.
 int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const AttnDesc& a, int kv_row0, int n_heads, int n_splits, void* o,
-                        float* o_part, float* lse_part, int* err, cudaStream_t s);
+                        float* o_part, float* lse_part, const Guard& gd, cudaStream_t s);
 
 }  // namespace sfm

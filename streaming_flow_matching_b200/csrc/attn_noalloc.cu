@@ -13,9 +13,13 @@
 // library holds it (SFM_NOALLOC_SCRATCH_BYTES) until the process exits.  In
 // host code its name is only a host-side stand-in, never a device address:
 // the first call on each device, with that device current, resolves the real
-// address with cudaGetSymbolAddress and keeps it.  All calls share the array
-// and it keeps the last call's contents; nothing in it has to start at zero,
-// because every partial the merge reads is written earlier in the same call.
+// address with cudaGetSymbolAddress and keeps it for that device's context (a
+// cudaDeviceReset brings up a new context, with the module loaded again, and
+// the next call resolves the address again).  All calls share the array and it
+// keeps the last call's contents; nothing in it has to start at zero, because
+// every partial the merge reads is written earlier in the same call.  A bounded
+// wait that gives up inside the kernel is reported, like for every standalone
+// call, through the per-device word sfm_check_call_error reads.
 #include <mutex>
 
 #include "attn.cuh"
@@ -28,22 +32,32 @@ static __device__ __align__(256) unsigned char g_attn_scratch[SFM_NOALLOC_SCRATC
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_scratch_dev[kMaxDevices] = {};
+struct ScratchSlot {
+  void* ctx = nullptr;   // the context the address belongs to
+  void* ptr = nullptr;
+};
+ScratchSlot g_scratch_dev[kMaxDevices];
 
-// Device address of g_attn_scratch on the current device (resolved once per device).
+// Device address of g_attn_scratch on the current device (resolved once per
+// device and context).
 int scratch_on_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return sfm::record_cuda(e);
   if (dev < 0 || dev >= kMaxDevices) return SFM_EUNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_dev[dev]) {
+  void* ctx = nullptr;
+  if (sfm::current_context(&ctx)) return SFM_ECUDA;
+  ScratchSlot& slot = g_scratch_dev[dev];
+  if (!ctx || slot.ctx != ctx || !slot.ptr) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_attn_scratch);
     if (e != cudaSuccess || !p) return sfm::record_cuda(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
-    g_scratch_dev[dev] = p;
+    if (!ctx && (sfm::current_context(&ctx) || !ctx)) return SFM_ECUDA;
+    slot.ctx = ctx;
+    slot.ptr = p;
   }
-  *out = g_scratch_dev[dev];
+  *out = slot.ptr;
   return SFM_OK;
 }
 

@@ -72,6 +72,8 @@ struct Args {
   float* o_part;               // [n_splits][total_rows][H][D]
   float* lse_part;             // [n_splits][total_rows][H]
   int* err;
+  unsigned long long wait_ns;  // bound of every wait
+  int fault;                   // SFM_FAULT_ATTN_NO_LOADS: the producer issues no loads (test only)
 };
 
 // 10 warps: two of the four SM sub-partitions hold three warps, which caps a
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0 && T > 0) {
+    if (lane == 0 && T > 0 && !(args.fault & SFM_FAULT_ATTN_NO_LOADS)) {
       // ---------------- TMA producer ----------------
       int kp[KST], vp[VST];               // parity of the last load into each stage
       for (int i = 0; i < KST; ++i) kp[i] = -1;
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       auto load_k = [&](int i) -> bool {   // i: tile index relative to t0
         const int s = i % KST;
         const uint32_t par = (uint32_t)((i / KST) & 1);
-        if (!mbar_wait(&k_empty[s], par ^ 1u, abort, args.err, 0x201)) return false;
+        if (!mbar_wait(&k_empty[s], par ^ 1u, abort, args.err, 0x201, args.wait_ns)) return false;
         const int krow = args.kv_row0 + (int)(kbase + (long long)(t0 + i) * BKV);
         mbar_arrive_expect_tx(&k_full[s], TILE);
         tma_load_3d(base + OFF_K + s * TILE, &map_k, &k_full[s], 0, h, krow);
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       auto load_v = [&](int i) -> bool {
         const int s = i % VST;
         const uint32_t par = (uint32_t)((i / VST) & 1);
-        if (!mbar_wait(&v_empty[s], par ^ 1u, abort, args.err, 0x202)) return false;
+        if (!mbar_wait(&v_empty[s], par ^ 1u, abort, args.err, 0x202, args.wait_ns)) return false;
         const int krow = args.kv_row0 + (int)(kbase + (long long)(t0 + i) * BKV);
         mbar_arrive_expect_tx(&v_full[s], TILE);
         tma_load_3d(base + OFF_V + s * TILE, &map_v, &v_full[s], 0, h, krow);
@@ -187,11 +189,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (ok && j + 2 < T) ok = load_k(j + 2);
       }
       if (!ok) {   // unwinding: let issued loads land before the CTA exits
-        mbar_drain(q_full, 0);
+        mbar_drain(q_full, 0, args.wait_ns);
         for (int i = 0; i < KST; ++i)
-          if (kp[i] >= 0) mbar_drain(&k_full[i], (uint32_t)kp[i]);
+          if (kp[i] >= 0) mbar_drain(&k_full[i], (uint32_t)kp[i], args.wait_ns);
         for (int i = 0; i < VST; ++i)
-          if (vp[i] >= 0) mbar_drain(&v_full[i], (uint32_t)vp[i]);
+          if (vp[i] >= 0) mbar_drain(&v_full[i], (uint32_t)vp[i], args.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ---------------- MMA issuer ----------------
       constexpr uint32_t idesc_s = idesc_bf16(BQ, BKV, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(BQ, D, false, true);
-      bool ok = mbar_wait(q_full, 0, abort, args.err, 0x203), issued = false;
+      bool ok = mbar_wait(q_full, 0, abort, args.err, 0x203, args.wait_ns), issued = false;
       auto issue_s = [&](int t, int ks) {   // S_t = Q_t K^T from K stage ks
         const uint32_t qa = base + OFF_Q + t * TILE, ka = base + OFF_K + ks * TILE;
         const uint32_t d = tmem + (uint32_t)(t * 256);
@@ -213,7 +215,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma_commit(&s_full[t]);
         issued = true;
       };
-      if (ok && (ok = mbar_wait(&k_full[0], 0, abort, args.err, 0x204))) {
+      if (ok && (ok = mbar_wait(&k_full[0], 0, abort, args.err, 0x204, args.wait_ns))) {
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
@@ -225,13 +227,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int vs = j % VST;
         const bool more = j + 1 < T;
         const int ks = (j + 1) % KST;
-        if (!mbar_wait(&v_full[vs], (uint32_t)((j / VST) & 1), abort, args.err, 0x206)) {
+        if (!mbar_wait(&v_full[vs], (uint32_t)((j / VST) & 1), abort, args.err, 0x206, args.wait_ns)) {
           ok = false;
           break;
         }
         const uint32_t va = base + OFF_V + vs * TILE;
         for (int t = 0; t < QT && ok; ++t) {
-          if (!mbar_wait(&p_full[t], (uint32_t)(j & 1), abort, args.err, 0x205)) {
+          if (!mbar_wait(&p_full[t], (uint32_t)(j & 1), abort, args.err, 0x205, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -248,12 +250,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (t == QT - 1) umma_commit(&v_empty[vs]);
           if (more) {
             if (t == 0 &&
-                !mbar_wait(&k_full[ks], (uint32_t)(((j + 1) / KST) & 1), abort, args.err, 0x204)) {
+                !mbar_wait(&k_full[ks], (uint32_t)(((j + 1) / KST) & 1), abort, args.err, 0x204, args.wait_ns)) {
               ok = false;
               break;
             }
             // S_t(j+1) overwrites P_t(j): wait until O_t's P V of this tile has completed
-            if (!mbar_wait(&o_done[t], (uint32_t)(j & 1), abort, args.err, 0x20B)) {
+            if (!mbar_wait(&o_done[t], (uint32_t)(j & 1), abort, args.err, 0x20B, args.wait_ns)) {
               ok = false;
               break;
             }
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (!ok && issued) {
         umma_commit(drain);
-        mbar_drain(drain, 0);
+        mbar_drain(drain, 0, args.wait_ns);
       }
     }
   } else {
@@ -283,7 +285,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = true;
     const float sc = args.scale_log2;
     for (int j = 0; j < T && ok; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], (uint32_t)(j & 1), abort, args.err, 0x207))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], (uint32_t)(j & 1), abort, args.err, 0x207, args.wait_ns))) {
         ok = false;
         break;
       }
@@ -409,7 +411,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // zero the V rows of the partial tile past the key range once the tile has
         // landed (tile A's warps; both P V products are issued after tile A's P is ready)
         const int vs = j % VST;
-        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[vs], (uint32_t)((j / VST) & 1), abort, args.err, 0x209))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&v_full[vs], (uint32_t)((j / VST) & 1), abort, args.err, 0x209, args.wait_ns))) {
           ok = false;
           break;
         }
@@ -431,7 +433,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     // ---- output ----
     if (ok && T > 0) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], (uint32_t)((T - 1) & 1), abort, args.err, 0x20A))) ok = false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], (uint32_t)((T - 1) & 1), abort, args.err, 0x20A, args.wait_ns))) ok = false;
       tc_fence_after();
     }
     const long long grow = row0 + t * BQ + r;
@@ -586,7 +588,7 @@ int attention_tc_splits_batch(const AttnDesc& a, int n_heads, int sms) {
 // q: map over [rows][H][128]; k, v: maps over the key rows ([rows][H][128]).
 int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const AttnDesc& a, int kv_row0, int n_heads, int n_splits, void* o,
-                        float* o_part, float* lse_part, int* err, cudaStream_t s) {
+                        float* o_part, float* lse_part, const Guard& gd, cudaStream_t s) {
   const long long total_rows = (long long)a.n * a.rows_per;
   if (total_rows == 0) return SFM_OK;
   atc::Args args{};
@@ -600,7 +602,9 @@ int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   args.o = (__nv_bfloat16*)o;
   args.o_part = o_part;
   args.lse_part = lse_part;
-  args.err = err;
+  args.err = gd.err;
+  args.wait_ns = gd.wait_ns;
+  args.fault = gd.fault;
   dim3 grid(a.n * args.qtiles, n_heads, n_splits);
   cudaFuncSetAttribute(atc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, atc::SMEM);
   int rc;

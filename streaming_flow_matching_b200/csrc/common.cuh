@@ -25,6 +25,17 @@ struct BatchDesc {
   long long base[kMaxBatch]; // first pool row of each session's region
   int valid[kMaxBatch];      // S_c: valid cached tokens
   long long p0[kMaxBatch];   // position of the unit's first token
+  int per_tau;               // 1: entry i is at flow time tau[i] (else one tau per call)
+  float tau[kMaxBatch];
+};
+
+// Bounded-wait settings of the tensor-core kernels: the device word in which a
+// timed-out wait records its site, the bound of every wait (1 s unless a test
+// shortens it), and the test-only fault (SFM_FAULT_* bits) to inject.
+struct Guard {
+  int* err = nullptr;
+  unsigned long long wait_ns = 1000000000ull;
+  int fault = 0;
 };
 
 struct Session {
@@ -35,6 +46,9 @@ struct Session {
 };
 
 int record_cuda(cudaError_t e);  // stores e for sfm_last_cuda_error; returns SFM_ECUDA or SFM_OK
+// The calling thread's current CUDA context (CUcontext, NULL before the runtime has
+// brought one up), through the driver entry point the runtime exposes.
+int current_context(void** ctx);
 void count_launch();             // one more kernel launched by this library
 
 // Records a CUDA event pair around the launches in its scope when the
@@ -56,9 +70,12 @@ class ProfScope {
 };
 
 // Launch helpers (each returns 0 / SFM_ECUDA after checking cudaGetLastError).
+// src_row_bytes / src_off_bytes: bytes per source row and offset of the copied
+// part inside it (0, 0: the source rows are exactly the cache rows).
 int launch_kv_append(const void* k, const void* v, void* k_pool, void* v_pool, int n_layers,
                      long long pool_tokens, int row_bytes, int n_tok, int unit_tokens,
-                     long long base_row, long long first_unit, int cache_units, cudaStream_t s);
+                     long long base_row, long long first_unit, int cache_units, cudaStream_t s,
+                     int src_row_bytes = 0, int src_off_bytes = 0);
 int launch_kv_read(const void* k_pool, const void* v_pool, void* k_dst, void* v_dst, int layer,
                    long long pool_tokens, int row_bytes, long long row0, long long n_rows,
                    cudaStream_t s);

@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int kblocks = args.K / BK;
   const int ksp = args.k_splits > 1 ? args.k_splits : 1;
   const int units_total = tiles * ksp;       // (tile, k slice) work units
+  const unsigned long long wait_ns = args.wait_ns ? args.wait_ns : kWaitNs;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
+    if (lane == 0 && !(args.fault & SFM_FAULT_GEMM_NO_LOADS)) {
       // ---------------- TMA producer (its own A rows and B rows) ----------------
       int s = 0;
       uint32_t ph = 0;
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int m0 = (t % m_tiles) * TM + (int)rank * BM;
         const int n0 = (t / m_tiles) * BN + (int)rank * C::B_ROWS;
         for (int kb = sl * kblocks / ksp; kb < (sl + 1) * kblocks / ksp; ++kb) {
-          if (!mbar_wait(&empty[s], ph ^ 1u, abort, args.err, 0x101)) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort, args.err, 0x101, wait_ns)) {
             ok = false;
             break;
           }
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         } else {
           for (int i = 0; i < C::STAGES; ++i)
-            if (last_parity[i] >= 0) mbar_drain(&full[i], (uint32_t)last_parity[i]);
+            if (last_parity[i] >= 0) mbar_drain(&full[i], (uint32_t)last_parity[i], wait_ns);
         }
       }
     }
@@ -196,15 +197,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int u = unit; u < units_total && ok; u += n_units) {
         const int sl = u / tiles;
         const int kb0 = sl * kblocks / ksp, kb1 = (sl + 1) * kblocks / ksp;
-        if (!(PAIR ? mbar_wait_cluster(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102)
-                   : mbar_wait(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102))) {
+        if (!(PAIR ? mbar_wait_cluster(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102, wait_ns)
+                   : mbar_wait(&acc_empty[acc], acc_ph ^ 1u, abort, args.err, 0x102, wait_ns))) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * C::ACC_COLS);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[s], ph, abort, args.err, 0x103)) {
+          if (!mbar_wait(&full[s], ph, abort, args.err, 0x103, wait_ns)) {
             ok = false;
             break;
           }
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           umma_commit_pair(drain, 1);
         else
           umma_commit(drain);
-        mbar_drain(drain, 0);
+        mbar_drain(drain, 0, wait_ns);
       }
     }
   } else {
@@ -287,8 +288,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t2 = 0; t2 < args.ss_n; ++t2) ss += args.ss_in[(size_t)row * args.ss_ld + t2];
         rinv = rsqrtf(ss / (float)args.norm_d + args.norm_eps);
       }
-      if (!__all_sync(0xffffffffu, PAIR ? mbar_wait_cluster(&acc_full[acc], acc_ph, abort, args.err, 0x104)
-                                        : mbar_wait(&acc_full[acc], acc_ph, abort, args.err, 0x104)))
+      if (!__all_sync(0xffffffffu, PAIR ? mbar_wait_cluster(&acc_full[acc], acc_ph, abort, args.err, 0x104, wait_ns)
+                                        : mbar_wait(&acc_full[acc], acc_ph, abort, args.err, 0x104, wait_ns)))
         break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);

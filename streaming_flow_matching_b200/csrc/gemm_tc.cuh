@@ -12,6 +12,8 @@ struct GemmArgs {
   void* C;               // output (EPI_F32 / EPI_STORE / EPI_GELU) or fp32 residual (EPI_RESID)
   int ldc;
   int* err;              // device error word (bounded-wait timeouts)
+  unsigned long long wait_ns;   // bound of every wait (0: 1 s)
+  int fault;             // SFM_FAULT_GEMM_NO_LOADS: the producers issue no loads (test only)
   // EPI_QKV
   const float* cos_t;    // [M][64]
   const float* sin_t;

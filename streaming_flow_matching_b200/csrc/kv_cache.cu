@@ -6,7 +6,9 @@
 // pre-sharded local cache).  Unit u goes to ring slot u mod cache_units.
 //
 // Layout: pool [L][pool_tokens][H * D_h]; a session owns rows
-// [base, base + cache_units * T_u + N).  Source slice [L][n_tok][H * D_h].
+// [base, base + cache_units * T_u + N).  Source slice [L][n_tok][H_src * D_h]:
+// a row of the slice may hold more heads than the cache (a rank of a
+// head-sharded cache copies its own head range of the broadcast slice).
 // Pure HBM copy: one CTA per (layer, token) row of K and V, 16-byte
 // streaming loads/stores (the slice is read once and the destination is not
 // re-read before it leaves L2).
@@ -17,7 +19,8 @@ namespace sfm {
 __global__ void __launch_bounds__(256) kv_append_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, uint4* __restrict__ k_pool,
     uint4* __restrict__ v_pool, int n_tok, int unit_tokens, long long pool_tokens, int row_vecs,
-    long long base_row, long long first_unit, int cache_units) {
+    int src_row_vecs, int src_off_vecs, long long base_row, long long first_unit,
+    int cache_units) {
   const long long src_row = blockIdx.x;                 // = layer * n_tok + t
   const int layer = (int)(src_row / n_tok);
   const int t = (int)(src_row - (long long)layer * n_tok);
@@ -25,8 +28,8 @@ __global__ void __launch_bounds__(256) kv_append_kernel(
   const int t_in = t - unit * unit_tokens;
   const long long slot = (first_unit + unit) % cache_units;
   const long long dst_row = (long long)layer * pool_tokens + base_row + slot * unit_tokens + t_in;
-  const uint4* ks = k + src_row * row_vecs;
-  const uint4* vs = v + src_row * row_vecs;
+  const uint4* ks = k + src_row * src_row_vecs + src_off_vecs;
+  const uint4* vs = v + src_row * src_row_vecs + src_off_vecs;
   uint4* kd = k_pool + dst_row * row_vecs;
   uint4* vd = v_pool + dst_row * row_vecs;
   for (int c = threadIdx.x; c < row_vecs; c += blockDim.x) {
@@ -57,13 +60,15 @@ static int block_for(int row_vecs) {
 
 int launch_kv_append(const void* k, const void* v, void* k_pool, void* v_pool, int n_layers,
                      long long pool_tokens, int row_bytes, int n_tok, int unit_tokens,
-                     long long base_row, long long first_unit, int cache_units, cudaStream_t s) {
+                     long long base_row, long long first_unit, int cache_units, cudaStream_t s,
+                     int src_row_bytes, int src_off_bytes) {
   const int row_vecs = row_bytes / 16;
+  const int src_row_vecs = (src_row_bytes ? src_row_bytes : row_bytes) / 16;
   const long long rows = (long long)n_layers * n_tok;
   if (rows == 0) return SFM_OK;
   kv_append_kernel<<<(unsigned)rows, block_for(row_vecs), 0, s>>>(
       (const uint4*)k, (const uint4*)v, (uint4*)k_pool, (uint4*)v_pool, n_tok, unit_tokens,
-      pool_tokens, row_vecs, base_row, first_unit, cache_units);
+      pool_tokens, row_vecs, src_row_vecs, src_off_bytes / 16, base_row, first_unit, cache_units);
   return record_cuda(cudaGetLastError());
 }
 

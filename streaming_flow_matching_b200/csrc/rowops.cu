@@ -57,8 +57,13 @@ __global__ void __launch_bounds__(128) embed_kernel(
   const int half = d / 2;
   const int ii = ic < half ? ic : ic - half;
   const double w = pow(10000.0, -2.0 * (double)ii / (double)d);
-  const double ang = 1000.0 * (double)tau * w;
-  const float te = (float)(ic < half ? sin(ang) : cos(ang));
+  auto temb = [&](float t) {
+    const double ang = 1000.0 * (double)t * w;
+    return (float)(ic < half ? sin(ang) : cos(ang));
+  };
+  // one flow time per call, or (several units of a pass) one per batch entry
+  float te = b.per_tau ? 0.f : temb(tau);
+  int te_sess = -1;
   float wr[CL];
 #pragma unroll
   for (int c = 0; c < CL; ++c) wr[c] = c < c_lat ? to_f(w_in[(size_t)ic * c_lat + c]) : 0.f;
@@ -71,6 +76,10 @@ __global__ void __launch_bounds__(128) embed_kernel(
     if (r >= rows) break;
     const int sess = r / b.n_tok;
     const int j = r - sess * b.n_tok;
+    if (b.per_tau && sess != te_sess) {
+      te = temb(b.tau[sess]);
+      te_sess = sess;
+    }
     const float* zr = z.p[sess] + (size_t)j * c_lat;
     float acc = 0.f;
 #pragma unroll
@@ -478,7 +487,7 @@ __global__ void __launch_bounds__(kHeadThreads)
         const int sess = row / b.n_tok;
         const int j = row - sess * b.n_tok;
         float* zr = z.p[sess] + (size_t)j * c_lat + c0 + c;
-        *zr = fmaf(dtau, v, *zr);
+        if (dtau != 0.f) *zr = fmaf(dtau, v, *zr);   // a zero-length step only reports v
         if (v_out.p[sess]) v_out.p[sess][(size_t)j * c_lat + c0 + c] = v;
       }
     }

@@ -4,10 +4,10 @@
 // CTA-pair (cluster of two, cta_group::2) forms of allocation, MMA, commit and
 // TMA completion used by the GEMM.
 //
-// Every wait is bounded: after kWaitNs nanoseconds a waiter raises the CTA's
-// abort flag and the kernel's global error word, and the roles of the kernel
-// unwind (drain their own asynchronous work with bounded waits, free TMEM,
-// return) instead of spinning forever.
+// Every wait is bounded: after a limit (a kernel argument, kWaitNs = 1 s by
+// default) a waiter raises the CTA's abort flag and the kernel's global error
+// word, and the roles of the kernel unwind (drain their own asynchronous work
+// with bounded waits, free TMEM, return) instead of spinning forever.
 #pragma once
 
 #include <cuda.h>
@@ -58,18 +58,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete.  Returns
-// false when kWaitNs pass first (after raising *abort and recording `site` in
-// *err if it is still 0), or as soon as another role of the CTA has raised
-// *abort.  `site` identifies the wait (kernel << 8 | wait site).
+// false when `limit` nanoseconds pass first (after raising *abort and recording
+// `site` in *err if it is still 0), or as soon as another role of the CTA has
+// raised *abort.  `site` identifies the wait (kernel << 8 | wait site).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* err, int site = kErrTimeout) {
+                                          int* err, int site = kErrTimeout,
+                                          unsigned long long limit = kWaitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitNs) {
+      if (globaltimer() - t0 > limit) {
         *abort = 1;
         if (err) atomicCAS(err, 0, site);
         return false;
@@ -79,10 +80,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // A bounded wait used only while unwinding: no error is raised.
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity,
+                                           unsigned long long limit = kWaitNs) {
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(bar, parity))
-    if (globaltimer() - t0 > kWaitNs) return;
+    if (globaltimer() - t0 > limit) return;
 }
 
 // ---- TMA (tile mode, no multicast) ---------------------------------------------
@@ -296,14 +298,15 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_
 // mbar_wait for a barrier that the other CTA of the pair arrives on (acquire at
 // cluster scope); same bound and error reporting as mbar_wait
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                                  int* err, int site) {
+                                                  int* err, int site,
+                                                  unsigned long long limit = kWaitNs) {
   if (mbar_try_wait_acq_cluster(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_acq_cluster(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitNs) {
+      if (globaltimer() - t0 > limit) {
         *abort = 1;
         if (err) atomicCAS(err, 0, site);
         return false;

@@ -105,6 +105,15 @@ class Performer:
         L.check(L.lib.sfm_kvcache_append(self._h, session, _ptr(k), _ptr(v), n_tok, _stream()),
                 "sfm_kvcache_append")
 
+    def kvcache_append_heads(self, session, k, v, head0):
+        """Appends heads [head0, head0 + n_heads) of a slice whose rows hold more heads
+        (one rank's share of a head-sharded cache)."""
+        _need(k, self.dtype, "k")
+        _need(v, self.dtype, "v", k.shape)
+        L.check(L.lib.sfm_kvcache_append_heads(self._h, session, _ptr(k), _ptr(v), k.shape[1],
+                                               k.shape[2], head0, _stream()),
+                "sfm_kvcache_append_heads")
+
     def kvcache_read(self, session, layer, row0, n_rows):
         shp = (n_rows, self.shape["n_heads"], self.shape["head_dim"])
         k = torch.empty(shp, dtype=self.dtype, device="cuda")
@@ -165,6 +174,40 @@ class Performer:
         t = (C.c_float * len(taus))(*taus)
         L.check(L.lib.sfm_fm_solve_guided_batched(self._h, n, s, u, zp, t, len(taus), scale, vp,
                                                   _stream()), "sfm_fm_solve_guided_batched")
+
+    def velocity_units(self, session, zs, taus, v_outs=None, commit=False):
+        """Velocities of len(zs) consecutive units after the session's cache in one
+        block-causal pass (unit u sees the cache and units <= u); commit appends the
+        units' own K/V to the cache.  Returns the velocity tensors."""
+        n = len(zs)
+        if len(taus) != n:
+            raise ValueError("zs and taus differ in length")
+        for z in zs:
+            _need(z, torch.float32, "z", (self.n_tok, self.shape["c_lat"]))
+        if v_outs is None:
+            v_outs = [torch.empty_like(z) for z in zs]
+        for v in v_outs:
+            _need(v, torch.float32, "v_out", (self.n_tok, self.shape["c_lat"]))
+        zp = (C.c_void_p * n)(*[z.data_ptr() for z in zs])
+        vp = (C.c_void_p * n)(*[v.data_ptr() for v in v_outs])
+        t = (C.c_float * n)(*taus)
+        L.check(L.lib.sfm_velocity_units(self._h, session, n, zp, t, vp, 1 if commit else 0,
+                                         _stream()), "sfm_velocity_units")
+        return v_outs
+
+    def plan(self):
+        """The projections' launch plan fixed at create (QKV, O, MLP-up, MLP-down)."""
+        p = L.sfm_plan()
+        L.check(L.lib.sfm_get_plan(self._h, C.byref(p)), "sfm_get_plan")
+        return {"block_n": list(p.block_n), "pair": list(p.pair), "k_splits": list(p.k_splits),
+                "fused_norm": p.fused_norm}
+
+    def test_fault(self, faults, wait_ns=0):
+        """Test-only: fault bits and wait bound of this handle's kernels (0, 0 = normal)."""
+        L.check(L.lib.sfm_test_fault(self._h, faults, wait_ns), "sfm_test_fault")
+
+    def clear_device_error(self):
+        L.check(L.lib.sfm_clear_device_error(self._h), "sfm_clear_device_error")
 
     def fm_solve_exact_velocity(self, z0, z, taus):
         """Test-only: the Euler solve with the exact rectified-flow velocity (z - z0) / tau

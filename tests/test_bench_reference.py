@@ -11,7 +11,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _run(rank):
     env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
     return subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny-fp32",
-                           "--steps", "1", "--warmup", "0", "--cpu-budget-s", "1"],
+                           "--steps", "1", "--warmup", "0"],
                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
 
 
@@ -27,7 +27,11 @@ def test_reference_arm_rank0_prints_one_line():
         assert k in d, k
     assert d["impl"] == "reference" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == os.cpu_count()
+    # the line says what it timed: a bounded sample of layers, extrapolated to a step
+    assert d["extrapolated"] is True and d["cpu_baseline"]["extrapolated"] is True
+    assert d["timed_layers"] == d["cpu_baseline"]["timed_layers"] == 1
+    assert d["measured_wall_s"] > 0 and d["cpu_baseline"]["threads"] >= 1
 
 
 def test_reference_arm_other_ranks_exit_quietly():

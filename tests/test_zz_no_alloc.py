@@ -37,23 +37,29 @@ def _allocating(q, k, v, dtype):
 
 
 def test_noalloc_matches_allocating_entry_point_on_consecutive_calls(cuda_device):
-    # a split-KV shape (uses the scratch array), then a smaller one, then the first again:
-    # stale contents of the shared array must not leak into a later call
-    cases = [(924, 17724, 24, "bf16"), (204, 704, 3, "bf16"), (924, 17724, 24, "bf16"),
-             (68, 452, 4, "fp32")]
-    used_scratch = False
+    # split-KV shapes (they use the scratch array) with different split counts, so a
+    # merge reads a different-sized part of what the previous call left there; then
+    # the first shape again, and an fp32 call that needs no scratch at all: stale
+    # contents of the shared array must not leak into a later call
+    cases = [(924, 17724, 24, "bf16"), (128, 20000, 2, "bf16"), (924, 17724, 24, "bf16"),
+             (512, 9000, 8, "bf16"), (204, 704, 3, "bf16"), (68, 452, 4, "fp32")]
+    splits = set()
     for n_q, n_kv, H, dt in cases:
         dtype = L.SFM_DTYPE_BF16 if dt == "bf16" else L.SFM_DTYPE_FP32
         q, k, v = S.make_qkv(n_q, n_kv, H, 128 if dt == "bf16" else 64, dtype=dt, device="cuda",
                              seed=n_kv)
         ref, need = _allocating(q, k, v, dtype)
-        used_scratch |= need > 0
+        if dt == "bf16":
+            # the partials of every split: [splits][n_q][H][128 + 1] fp32
+            assert need > 0 and need % (n_q * H * 129 * 4) == 0, (n_q, n_kv, H, need)
+            splits.add(need // (n_q * H * 129 * 4))
         o = torch.full_like(q, float("nan"))
         assert _noalloc(q, k, v, o, dtype) == L.SFM_OK
         torch.cuda.synchronize()
         e = rel_l2(o.float().cpu().numpy(), ref.float().cpu().numpy())
         assert e <= (BF16_TOL if dt == "bf16" else FP32_TOL), (n_q, n_kv, H, e)
-    assert used_scratch
+    assert len(splits) >= 3, splits
+    assert L.check_call_error() == 0
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_device):

@@ -121,6 +121,16 @@ def make_kv_slices(w: Workload, n_units, device="cpu", seed=SEED_CACHE):
     return _normal(g, shape, 1.0, dt, device), _normal(g, shape, 1.0, dt, device)
 
 
+def make_kv_layer(w: Workload, n_units, layer, device="cpu", seed=SEED_CACHE):
+    """One layer of the thinker's K/V slices, drawn from its own generator (seed
+    1000 * seed + layer), so a 28-layer cache can be built one layer at a time
+    without holding every layer's fp32 draw: K, V each [n_units*T_u][H][D]."""
+    dt = torch_dtype(w.dtype)
+    g = _gen(1000 * seed + layer, device)
+    shape = (n_units * w.unit_kv_tokens, w.n_heads, w.head_dim)
+    return _normal(g, shape, 1.0, dt, device), _normal(g, shape, 1.0, dt, device)
+
+
 def make_latents(w: Workload, device="cpu", n_sessions=1):
     """Clean latents z0 (seed 3) and noise eps (seed 4), fp32 [S][N][C]."""
     shape = (n_sessions, w.n_tokens, w.c_lat)

@@ -115,3 +115,30 @@ def test_full_size_append_wraps_into_slot_zero(cuda_device):
     info = p.session_info(s)
     assert info["units_appended"] == 49 and info["valid_tokens"] == 57600 and info["p0"] == 49 * T
     p.close()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_sharded_append_takes_each_ranks_head_range(cuda_device, world):
+    # each rank of a head-sharded cache (Ulysses group of `world` ranks) keeps heads
+    # [r H / P, (r + 1) H / P) of the broadcast slice, bit for bit, ring included
+    from streaming_flow_matching_b200.ulysses import UlyssesPlan, cache_heads
+    w = W.replace(n_heads=4)
+    n_units, cap = 5, 3
+    k, v = S.make_kv_slices(w, n_units)
+    plan = UlyssesPlan(w.n_video, w.n_audio, w.n_heads, world)
+    for r in range(world):
+        wr = w.replace(n_heads=plan.heads_per_rank)
+        ref = O.KVCache(w.n_layers, cap, w.unit_kv_tokens, wr.n_heads, w.head_dim)
+        ref.append(O.f64(cache_heads(plan, k, r)), O.f64(cache_heads(plan, v, r)))
+        p = _perf(wr, cap)
+        s = p.open_session(cap)
+        h0, _ = plan.head_range(r)
+        p.kvcache_append_heads(s, k.cuda(), v.cuda(), h0)
+        torch.cuda.synchronize()
+        gk, gv = _read_all(p, s, wr, cap)
+        assert np.array_equal(O.f64(gk), ref.k) and np.array_equal(O.f64(gv), ref.v)
+        assert p.session_info(s)["units_appended"] == n_units
+        # a head range past the slice's heads is refused before any launch
+        with pytest.raises(Exception):
+            p.kvcache_append_heads(s, k.cuda(), v.cuda(), w.n_heads - plan.heads_per_rank + 1)
+        p.close()

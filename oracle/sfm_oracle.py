@@ -75,6 +75,9 @@ class Config:
     unit_kv_tokens: int
     rope_theta: float = 10000.0
     rms_eps: float = 1e-6
+    mlp: str = "gelu"          # "gelu" | "swiglu" (open reading, see swiglu_mlp)
+    rope_mode: str = "1d"      # "1d" | "3d" (open reading, see rope_3d)
+    grid_w: int = 0            # 3-D RoPE: video raster width in tokens
 
     @property
     def n_tokens(self) -> int:
@@ -123,6 +126,85 @@ def rope(x, pos, theta):
     a = x[..., :half]
     b = x[..., half:]
     return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def rope_3d_bands(head_dim):
+    """Pair bands of the 3-D rotary embedding: (pairs of t, pairs of y, pairs of x).
+
+    Each spatial axis takes head_dim // 6 of the head_dim / 2 rotate-half pairs and time
+    takes the rest (128 dims: 22 + 21 + 21 pairs), the split of the Wan video models."""
+    half = head_dim // 2
+    ns = head_dim // 6
+    return half - 2 * ns, ns, ns
+
+
+def rope_3d(x, pos3, theta):
+    """3-D rotary embedding over (t, y, x), rotate-half pairing (i, i + D/2).
+
+    x: [N][H][D]; pos3: [N][3] integer positions (t, y, x).  Pair i of band b (time,
+    rows, columns) with n_b pairs, k = i - start_b, rotates by pos3[:, b] * theta^(-k / n_b):
+    the 1-D frequency ladder restarted per axis over the band's own width.
+    """
+    x = f64(x)
+    d = x.shape[-1]
+    half = d // 2
+    nt, ny, nx = rope_3d_bands(d)
+    pos3 = np.asarray(pos3, dtype=np.float64)
+    axis = np.concatenate([np.zeros(nt, int), np.ones(ny, int), np.full(nx, 2)])
+    k = np.concatenate([np.arange(nt), np.arange(ny), np.arange(nx)]).astype(np.float64)
+    nb = np.concatenate([np.full(nt, nt), np.full(ny, ny), np.full(nx, nx)]).astype(np.float64)
+    w = theta ** (-k / nb)
+    ang = pos3[:, axis] * w[None, :]                  # [N][half]
+    c = np.cos(ang)[:, None, :]
+    sn = np.sin(ang)[:, None, :]
+    a = x[..., :half]
+    b = x[..., half:]
+    return np.concatenate([a * c - b * sn, b * c + a * sn], axis=-1)
+
+
+def token_positions(cfg, p0, n_units=1):
+    """Positions of n_units consecutive units starting at token position p0 (1-D: p0 + i)
+    or, for 3-D RoPE, (t, y, x) per token: t = the unit's index on the timeline
+    (p0 // unit_kv_tokens + u), (y, x) the video token's raster cell, (0, 0) for audio."""
+    n = cfg.n_tokens
+    if cfg.rope_mode == "1d":
+        return p0 + np.arange(n_units * n)
+    j = np.arange(n)
+    y = np.where(j < cfg.n_video, j // max(cfg.grid_w, 1), 0)
+    x = np.where(j < cfg.n_video, j % max(cfg.grid_w, 1), 0)
+    t0 = p0 // cfg.unit_kv_tokens
+    return np.concatenate([np.stack([np.full(n, t0 + u), y, x], axis=1) for u in range(n_units)])
+
+
+def apply_rope(cfg, x, pos):
+    """The rotary embedding of the configuration: 1-D over positions, or 3-D over (t, y, x)."""
+    if cfg.rope_mode == "3d":
+        return rope_3d(x, pos, cfg.rope_theta)
+    return rope(x, pos, cfg.rope_theta)
+
+
+def silu(x):
+    """SiLU: x * sigmoid(x) = x / (1 + exp(-x))."""
+    x = f64(x)
+    return x / (1.0 + np.exp(-x))
+
+
+def swiglu_gate_up(cfg, w1):
+    """Gate and up matrices [F][d] of a SwiGLU W_1 stored [2F][d] in interleaved blocks of
+    64 rows: rows 128 b + [0, 64) are gate rows 64 b + [0, 64), rows 128 b + [64, 128) the
+    matching up rows (the layout the library reads)."""
+    w1 = f64(w1)
+    blocks = w1.reshape(-1, 2, 64, w1.shape[-1])
+    return blocks[:, 0].reshape(-1, w1.shape[-1]), blocks[:, 1].reshape(-1, w1.shape[-1])
+
+
+def mlp_forward(cfg, h, lw):
+    """The block's MLP on normalised rows h: tanh-GELU (W_1 [F][d]) or SwiGLU
+    (silu(h W_g^T) * (h W_u^T), W_1 [2F][d] as in swiglu_gate_up), then W_2."""
+    if cfg.mlp == "swiglu":
+        wg, wu = swiglu_gate_up(cfg, lw["w_1"])
+        return linear(silu(linear(h, wg)) * linear(h, wu), lw["w_2"])
+    return linear(gelu_tanh(linear(h, lw["w_1"])), lw["w_2"])
 
 
 def tau_embedding(tau, d):
@@ -253,14 +335,14 @@ def layer_forward(cfg: Config, x, lw, k_ctx, v_ctx, pos, visible=None, return_kv
     q = qkv[:, :hd].reshape(n, cfg.n_heads, cfg.head_dim)
     k = qkv[:, hd:2 * hd].reshape(n, cfg.n_heads, cfg.head_dim)
     v = qkv[:, 2 * hd:].reshape(n, cfg.n_heads, cfg.head_dim)
-    q = rope(q, pos, cfg.rope_theta)
-    k = rope(k, pos, cfg.rope_theta)
+    q = apply_rope(cfg, q, pos)
+    k = apply_rope(cfg, k, pos)
     K = np.concatenate([f64(k_ctx), k], axis=0)
     V = np.concatenate([f64(v_ctx), v], axis=0)
     a = attention(q, K, V, visible)
     x = x + linear(a.reshape(n, hd), lw["w_o"])
     h2 = rmsnorm(x, lw["g_mlp"], cfg.rms_eps)
-    x = x + linear(gelu_tanh(linear(h2, lw["w_1"])), lw["w_2"])
+    x = x + mlp_forward(cfg, h2, lw)
     if return_kv:
         return x, k, v
     return x
@@ -283,7 +365,7 @@ def f_theta(cfg: Config, z, tau, w, cache_k, cache_v, valid_tokens, p0, pos=None
     """
     x = embed(cfg, z, tau, w, modality)
     if pos is None:
-        pos = p0 + np.arange(cfg.n_tokens)
+        pos = token_positions(cfg, p0)
     for li, lw in enumerate(w["layers"]):
         kc = f64(cache_k[li][:valid_tokens])
         vc = f64(cache_v[li][:valid_tokens])
@@ -378,7 +460,7 @@ def f_theta_sequence(cfg: Config, zs, taus, w, return_kv=False):
     n_units = len(zs)
     x = np.concatenate([embed(cfg, zs[u], taus[u], w) for u in range(n_units)], axis=0)
     units = np.repeat(np.arange(n_units), n)
-    pos = np.arange(n_units * n)
+    pos = token_positions(cfg, 0, n_units)
     visible = block_causal_visible(units, units)
     kv = []
     empty = np.zeros((0, cfg.n_heads, cfg.head_dim))
@@ -408,7 +490,7 @@ def f_theta_units(cfg: Config, zs, taus, w, cache_k, cache_v, valid_tokens, p0, 
     n_units = len(zs)
     x = np.concatenate([embed(cfg, zs[u], taus[u], w) for u in range(n_units)], axis=0)
     units = np.repeat(np.arange(n_units), n)
-    pos = p0 + np.arange(n_units * n)
+    pos = token_positions(cfg, p0, n_units)
     key_units = np.concatenate([np.full(valid_tokens, -1), units])   # prefix = unit -1
     visible = block_causal_visible(units, key_units)
     kv = []

@@ -512,3 +512,115 @@ def test_guided_solve_matches_brute_force_velocities():
         vu = np.array(BF.velocity(cfg, zz, t, w, *uncond))
         zz = zz - 0.5 * (vu + s * (vc - vu))
     np.testing.assert_allclose(got, zz, rtol=1e-10, atol=1e-11)
+
+
+# --------------------------------------------------------------------------
+# open-reading variants: 3-D rotary embedding, SwiGLU MLP, 64-channel tokens
+# --------------------------------------------------------------------------
+
+def test_rope_3d_scalar_brute_force():
+    # D = 12: 6 rotate-half pairs, 2 per axis (t, y, x); pair k of an axis turns by
+    # pos_axis * theta^(-k / 2)
+    rng = np.random.default_rng(50)
+    x = rng.standard_normal((3, 2, 12))
+    pos3 = np.array([[3, 1, 2], [0, 4, 1], [7, 0, 0]])
+    theta = 100.0
+    got = O.rope_3d(x, pos3, theta)
+    assert O.rope_3d_bands(12) == (2, 2, 2)
+    for n in range(3):
+        for h in range(2):
+            for i in range(6):
+                ax, k = i // 2, i % 2
+                ang = pos3[n, ax] * theta ** (-k / 2.0)
+                a, b = x[n, h, i], x[n, h, i + 6]
+                assert abs(got[n, h, i] - (a * math.cos(ang) - b * math.sin(ang))) < 1e-12
+                assert abs(got[n, h, i + 6] - (b * math.cos(ang) + a * math.sin(ang))) < 1e-12
+
+
+def test_rope_3d_bands_and_relative_positions():
+    assert O.rope_3d_bands(128) == (22, 21, 21)        # the Wan split of 64 pairs
+    assert O.rope_3d_bands(64) == (12, 10, 10)
+    rng = np.random.default_rng(51)
+    q = rng.standard_normal((1, 1, 128))
+    k = rng.standard_normal((1, 1, 128))
+    def dot(a, b):
+        return float((O.rope_3d(q, [a], 1e4) * O.rope_3d(k, [b], 1e4)).sum())
+    # depends on the position differences only, per axis
+    assert abs(dot((5, 2, 7), (3, 1, 1)) - dot((12, 6, 9), (10, 5, 3))) < 1e-9
+    assert abs(dot((5, 2, 7), (3, 1, 1)) - dot((5, 2, 7), (3, 2, 1))) > 1e-6
+    # rotations keep every pair's norm; (0, 0, 0) is the identity
+    y = O.rope_3d(q, [(9, 4, 33)], 1e4)
+    np.testing.assert_allclose(y[..., :64] ** 2 + y[..., 64:] ** 2, q[..., :64] ** 2 + q[..., 64:] ** 2,
+                               atol=1e-12)
+    np.testing.assert_array_equal(O.rope_3d(q, [(0, 0, 0)], 1e4), q)
+
+
+def test_token_positions_3d_raster_and_audio():
+    cfg = tiny_cfg(n_video=6, n_audio=2, unit_kv_tokens=8)
+    cfg.rope_mode, cfg.grid_w = "3d", 3
+    pos = O.token_positions(cfg, 16, n_units=2)           # p0 = 16 tokens = 2 units
+    assert pos.shape == (16, 3)
+    np.testing.assert_array_equal(pos[:8], [[2, 0, 0], [2, 0, 1], [2, 0, 2], [2, 1, 0], [2, 1, 1],
+                                            [2, 1, 2], [2, 0, 0], [2, 0, 0]])
+    np.testing.assert_array_equal(pos[8:, 0], [3] * 8)
+    cfg.rope_mode = "1d"
+    np.testing.assert_array_equal(O.token_positions(cfg, 16, n_units=2), 16 + np.arange(16))
+
+
+def test_silu_and_swiglu_layout():
+    x = np.linspace(-30, 30, 121)
+    np.testing.assert_allclose(O.silu(x), x * scipy.special.expit(x), rtol=1e-13, atol=1e-15)
+    assert O.silu(0.0) == 0.0 and abs(O.silu(40.0) - 40.0) < 1e-12
+    rng = np.random.default_rng(52)
+    wg = rng.standard_normal((128, 5))
+    wu = rng.standard_normal((128, 5))
+    w1 = np.concatenate([np.concatenate([wg[64 * b:64 * b + 64], wu[64 * b:64 * b + 64]]) for b in range(2)])
+    g, u = O.swiglu_gate_up(None, w1)
+    np.testing.assert_array_equal(g, wg)
+    np.testing.assert_array_equal(u, wu)
+
+
+def test_swiglu_mlp_brute_force():
+    cfg = tiny_cfg(d_mlp=64)
+    cfg.mlp = "swiglu"
+    rng = np.random.default_rng(53)
+    h = rng.standard_normal((3, cfg.d_model))
+    lw = {"w_1": rng.standard_normal((128, cfg.d_model)) * 0.3,
+          "w_2": rng.standard_normal((cfg.d_model, 64)) * 0.3}
+    got = O.mlp_forward(cfg, h, lw)
+    for r in range(3):
+        for o in range(cfg.d_model):
+            acc = 0.0
+            for f in range(64):
+                g = sum(h[r, c] * lw["w_1"][f, c] for c in range(cfg.d_model))        # gate rows 0..63
+                u = sum(h[r, c] * lw["w_1"][64 + f, c] for c in range(cfg.d_model))   # up rows 64..127
+                acc += g / (1.0 + math.exp(-g)) * u * lw["w_2"][o, f]
+            assert abs(got[r, o] - acc) < 1e-10
+
+
+@pytest.mark.parametrize("mlp,rope_mode", [("swiglu", "1d"), ("gelu", "3d"), ("swiglu", "3d")])
+def test_variant_performer_form_equals_block_causal_sequence(mlp, rope_mode):
+    # the performer form over a cache of earlier units' own K/V equals the masked
+    # full-sequence form with the variant MLP and rotary embedding too
+    cfg = tiny_cfg(unit_kv_tokens=5, d_mlp=64)
+    cfg.mlp, cfg.rope_mode, cfg.grid_w = mlp, rope_mode, 3
+    rng = np.random.default_rng(54)
+    w = tiny_weights(cfg, rng)
+    if mlp == "swiglu":
+        for lw in w["layers"]:
+            lw["w_1"] = rng.standard_normal((2 * cfg.d_mlp, cfg.d_model)) * 0.3
+    zs = [rng.standard_normal((cfg.n_tokens, cfg.c_lat)) for _ in range(3)]
+    taus = [0.0, 0.0, 0.6]
+    seq, kv = O.f_theta_sequence(cfg, zs, taus, w, return_kv=True)
+    n = cfg.n_tokens
+    ck = [kv[l][0][:2 * n] for l in range(cfg.n_layers)]
+    cv = [kv[l][1][:2 * n] for l in range(cfg.n_layers)]
+    got = O.f_theta(cfg, zs[2], taus[2], w, ck, cv, 2 * n, 2 * n)
+    np.testing.assert_allclose(got, seq[2], atol=1e-12)
+    units = O.f_theta_units(cfg, zs, taus, w, ck, cv, 0, 0)
+    for a, b in zip(units, seq):
+        np.testing.assert_allclose(a, b, atol=1e-12)
+    # the variant changes the result (it is not silently ignored)
+    cfg2 = tiny_cfg(unit_kv_tokens=5, d_mlp=64)
+    if mlp == "gelu":
+        assert np.max(np.abs(O.f_theta_sequence(cfg2, zs, taus, w)[2] - seq[2])) > 1e-6

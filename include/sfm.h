@@ -84,7 +84,26 @@ typedef struct sfm_config {
                             0: sfm_kvcache_append returns SFM_ECAPACITY          */
   double rope_theta;     /* RoPE base (10000)                                   */
   double rms_eps;        /* RMSNorm epsilon (1e-6)                              */
+  /* Variants the pages leave open (the defaults, 0, are the plain readings). */
+  int mlp;               /* SFM_MLP_GELU: x += GELU_tanh(h W_1^T) W_2^T, W_1 [F][d];
+                            SFM_MLP_SWIGLU: x += (silu(h W_g^T) * (h W_u^T)) W_2^T,
+                            W_1 [2F][d] holding W_g and W_u in interleaved blocks of
+                            64 rows (rows 128 b + [0, 64): gate rows 64 b + [0, 64);
+                            rows 128 b + [64, 128): the matching up rows); F % 64 == 0 */
+  int rope;              /* SFM_ROPE_1D: positions p0 + j;
+                            SFM_ROPE_3D: (t, y, x) per token -- t the unit's index on
+                            the timeline (units appended before it), (y, x) the video
+                            token's cell in a raster of grid_w columns, (0, 0) for
+                            audio; the head's D/2 rotate-half pairs split into
+                            D/2 - 2 (D/6) time pairs and D/6 pairs per spatial axis,
+                            each axis with its own frequency ladder theta^(-k / n_axis) */
+  int grid_w;            /* SFM_ROPE_3D: video raster width in tokens (>= 1)     */
 } sfm_config;
+
+#define SFM_MLP_GELU    0
+#define SFM_MLP_SWIGLU  1
+#define SFM_ROPE_1D     0
+#define SFM_ROPE_3D     1
 
 /*
  * Weights of f_theta: device pointers of the config's dtype, each 16-byte
@@ -98,6 +117,7 @@ typedef struct sfm_config {
  *   w_o    [d][H D_h]
  *   g_mlp  [d]              pre-MLP RMSNorm gain
  *   w_1    [F][d], w_2 [d][F]   x += GELU_tanh(RMSNorm(x) W_1^T) W_2^T
+ *                           (SwiGLU: w_1 [2F][d] in the interleaved layout above)
  * A handle created with w == NULL supports only the cache calls.
  */
 typedef struct sfm_weights {

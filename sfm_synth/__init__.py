@@ -43,6 +43,9 @@ class Workload:
     dtype: str               # "bf16" | "fp32"
     rope_theta: float = 10000.0
     rms_eps: float = 1e-6
+    mlp: str = "gelu"        # "gelu" | "swiglu": W_1 [F][d] or [2F][d] (interleaved gate/up)
+    rope: str = "1d"         # "1d" | "3d": positions p0 + j or (t, y, x)
+    grid_w: int = 0          # 3-D RoPE: video raster width in tokens
 
     @property
     def n_tokens(self):
@@ -107,7 +110,8 @@ def make_weights(w: Workload, device="cpu", seed=SEED_WEIGHTS):
             "w_qkv": _normal(g, (3 * w.hd, w.d_model), WEIGHT_STD, dt, device),
             "w_o": _normal(g, (w.d_model, w.hd), WEIGHT_STD, dt, device),
             "g_mlp": ones(w.d_model),
-            "w_1": _normal(g, (w.d_mlp, w.d_model), WEIGHT_STD, dt, device),
+            "w_1": _normal(g, ((2 if w.mlp == "swiglu" else 1) * w.d_mlp, w.d_model), WEIGHT_STD,
+                           dt, device),
             "w_2": _normal(g, (w.d_model, w.d_mlp), WEIGHT_STD, dt, device),
         })
     return out

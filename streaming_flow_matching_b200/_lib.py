@@ -16,6 +16,8 @@ SFM_OK, SFM_EINVAL, SFM_ECAPACITY, SFM_ESESSION, SFM_ECUDA, SFM_ENOMEM, SFM_EUNS
 SFM_EDEVICE = -7
 SFM_FAULT_NONE, SFM_FAULT_ATTN_NO_LOADS, SFM_FAULT_GEMM_NO_LOADS = 0, 1, 2
 SFM_DTYPE_BF16, SFM_DTYPE_FP32 = 0, 1
+SFM_MLP_GELU, SFM_MLP_SWIGLU = 0, 1
+SFM_ROPE_1D, SFM_ROPE_3D = 0, 1
 SFM_NOALLOC_SCRATCH_BYTES = 64 << 20
 SFM_LINEAR_F32, SFM_LINEAR_OUT, SFM_LINEAR_GELU, SFM_LINEAR_RESID = 0, 1, 2, 3
 
@@ -25,7 +27,8 @@ class sfm_config(C.Structure):
                 ("head_dim", C.c_int), ("d_mlp", C.c_int), ("c_lat", C.c_int),
                 ("n_video", C.c_int), ("n_audio", C.c_int), ("unit_kv_tokens", C.c_int),
                 ("max_sessions", C.c_int), ("pool_tokens", C.c_longlong), ("dtype", C.c_int),
-                ("ring", C.c_int), ("rope_theta", C.c_double), ("rms_eps", C.c_double)]
+                ("ring", C.c_int), ("rope_theta", C.c_double), ("rms_eps", C.c_double),
+                ("mlp", C.c_int), ("rope", C.c_int), ("grid_w", C.c_int)]
 
 
 _PP = C.POINTER(C.c_void_p)

@@ -51,6 +51,7 @@ struct sfm_handle {
   float* x = nullptr;        // [M][d] fp32 residual stream
   void* xn = nullptr;        // [M][d] normalised GEMM operand
   float* qkv32 = nullptr;    // [M][3 H D] fp32 projection output
+  float* mlp32 = nullptr;    // [M][2F] fp32 gate / up projection (fp32 SwiGLU)
   void* q = nullptr;         // [M][H][D] rotated queries
   void* ao = nullptr;        // [M][H D] attention output
   void* hmlp = nullptr;      // [M][F] GELU(MLP-up)
@@ -88,6 +89,10 @@ int validate_config(const sfm_config* c) {
       c->unit_kv_tokens < 1 || c->max_sessions < 1 || c->pool_tokens < 0)
     return SFM_EINVAL;
   if (c->dtype != SFM_DTYPE_BF16 && c->dtype != SFM_DTYPE_FP32) return SFM_EINVAL;
+  if (c->mlp != SFM_MLP_GELU && c->mlp != SFM_MLP_SWIGLU) return SFM_EINVAL;
+  if (c->rope != SFM_ROPE_1D && c->rope != SFM_ROPE_3D) return SFM_EINVAL;
+  if (c->rope == SFM_ROPE_3D && (c->grid_w < 1 || c->head_dim < 6)) return SFM_EINVAL;
+  if (c->mlp == SFM_MLP_SWIGLU && c->d_mlp % 64) return SFM_EUNSUPPORTED;
   if (!(c->rms_eps >= 0.0) || !(c->rope_theta > 0.0)) return SFM_EINVAL;
   if (c->max_sessions > kMaxBatch) return SFM_EUNSUPPORTED;
   if ((long long)c->n_layers * c->pool_tokens >= (1LL << 31)) return SFM_EUNSUPPORTED;
@@ -139,6 +144,7 @@ int fill_batch(const sfm_handle* h, int n, const int* sessions, BatchDesc* b) {
     b->base[i] = s.base_row;
     b->valid[i] = (int)valid_tokens(h, s);
     b->p0[i] = s.units * h->cfg.unit_kv_tokens;
+    b->t_unit[i] = s.units;
   }
   return SFM_OK;
 }
@@ -311,10 +317,15 @@ int run_step(sfm_handle* h, const BatchDesc& b, const AttnDesc& ad, float* const
     }
     {
       ProfScope ps(SFM_PROF_GEMM_UP, s);
+      const bool swiglu = c.mlp == SFM_MLP_SWIGLU;
       if (tc) {
         SFM_TRY(launch_gemm_tc(h->map_xn, h->map_w1[l],
-                               normed(gemm_args(M, F, d, EPI_GELU, h->hmlp, F, h->gd, h->bn_up, h->pair_up)),
+                               normed(gemm_args(M, swiglu ? 2 * F : F, d, swiglu ? EPI_SWIGLU : EPI_GELU,
+                                                h->hmlp, F, h->gd, h->bn_up, h->pair_up)),
                                h->sms, s));
+      } else if (swiglu) {
+        SFM_TRY(launch_gemm(h->xn, h->w_1[l], h->mlp32, M, 2 * F, d, EPI_F32, dt, s));
+        SFM_TRY(launch_swiglu(h->mlp32, h->hmlp, M, F, dt, s));
       } else {
         SFM_TRY(launch_gemm(h->xn, h->w_1[l], h->hmlp, M, F, d, EPI_GELU, dt, s));
       }
@@ -379,7 +390,8 @@ int solve_direct(sfm_handle* h, const Pass& ps, float* const* z, const float* ta
   int rc;
   {
     ProfScope prof(SFM_PROF_ROWOPS, s);
-    rc = launch_rope_table(ps.b, h->cos_t, h->sin_t, h->cfg.head_dim, h->cfg.rope_theta, s);
+    rc = launch_rope_table(ps.b, h->cos_t, h->sin_t, h->cfg.head_dim, h->cfg.rope_theta, s,
+                           h->cfg.rope == SFM_ROPE_3D, h->cfg.grid_w);
   }
   if (rc) return rc;
   for (int i = 0; i + 1 < n_taus; ++i) {
@@ -500,6 +512,8 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     if (!rc) rc = dalloc(h, &h->q, M * hd * es);
     if (!rc) rc = dalloc(h, &h->ao, M * hd * es);
     if (!rc) rc = dalloc(h, &h->hmlp, M * F * es);
+    if (!rc && cfg->mlp == SFM_MLP_SWIGLU && cfg->dtype == SFM_DTYPE_FP32)
+      rc = dalloc(h, &h->mlp32, M * 2 * F * 4);
     if (!rc) rc = dalloc(h, &h->cos_t, M * (cfg->head_dim / 2) * 4);
     if (!rc) rc = dalloc(h, &h->ss, M * ((cfg->d_model + 127) / 128) * 4);
     if (!rc) rc = dalloc(h, &h->sin_t, M * (cfg->head_dim / 2) * 4);
@@ -565,11 +579,13 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     const int mm = (int)M;
     h->pair_qkv = gemm_tc_pair(mm, 3 * hd_, hd_, EPI_QKV, h->sms);
     h->pair_o = gemm_tc_pair(mm, d_, 0, EPI_RESID, h->sms);
-    h->pair_up = gemm_tc_pair(mm, F_, 0, EPI_GELU, h->sms);
+    const bool swiglu = cfg->mlp == SFM_MLP_SWIGLU;
+    const int up_n = swiglu ? 2 * F_ : F_, up_epi = swiglu ? EPI_SWIGLU : EPI_GELU;
+    h->pair_up = gemm_tc_pair(mm, up_n, 0, up_epi, h->sms);
     h->pair_down = gemm_tc_pair(mm, d_, 0, EPI_RESID, h->sms);
     h->bn_qkv = gemm_tc_block_n(mm, 3 * hd_, hd_, EPI_QKV, h->sms, h->pair_qkv);
     h->bn_o = gemm_tc_block_n(mm, d_, 0, EPI_RESID, h->sms, h->pair_o);
-    h->bn_up = gemm_tc_block_n(mm, F_, 0, EPI_GELU, h->sms, h->pair_up);
+    h->bn_up = gemm_tc_block_n(mm, up_n, 0, up_epi, h->sms, h->pair_up);
     h->bn_down = gemm_tc_block_n(mm, d_, 0, EPI_RESID, h->sms, h->pair_down);
     if (!h->bn_qkv || !h->bn_o || !h->bn_up || !h->bn_down) rc = SFM_EUNSUPPORTED;
     if (!rc) {
@@ -583,7 +599,7 @@ int sfm_create(const sfm_config* cfg, const sfm_weights* w, sfm_handle** out) {
     for (int l = 0; l < L_ && !rc; ++l) {
       rc = make_b_map(&h->map_wqkv[l], h->w_qkv[l], 3 * hd_, d_, h->bn_qkv / (h->pair_qkv ? 2 : 1));
       if (!rc) rc = make_b_map(&h->map_wo[l], h->w_o[l], d_, hd_, h->bn_o / (h->pair_o ? 2 : 1));
-      if (!rc) rc = make_b_map(&h->map_w1[l], h->w_1[l], F_, d_, h->bn_up / (h->pair_up ? 2 : 1));
+      if (!rc) rc = make_b_map(&h->map_w1[l], h->w_1[l], up_n, d_, h->bn_up / (h->pair_up ? 2 : 1));
       if (!rc) rc = make_b_map(&h->map_w2[l], h->w_2[l], d_, F_, h->bn_down / (h->pair_down ? 2 : 1));
     }
   }
@@ -860,6 +876,7 @@ int sfm_velocity_units(sfm_handle* h, int session, int n_units, const float* con
     b.base[u] = se.base_row;
     b.valid[u] = (int)(valid + u * N);           // unit u's K/V rows follow the earlier units'
     b.p0[u] = se.units * T + u * N;
+    b.t_unit[u] = se.units + u;
     b.tau[u] = taus[u];
   }
   AttnDesc& a = ps.a;

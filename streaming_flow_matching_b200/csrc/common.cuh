@@ -27,6 +27,7 @@ struct BatchDesc {
   long long p0[kMaxBatch];   // position of the unit's first token
   int per_tau;               // 1: entry i is at flow time tau[i] (else one tau per call)
   float tau[kMaxBatch];
+  long long t_unit[kMaxBatch]; // the unit's index on the timeline (3-D rotary embedding)
 };
 
 // Bounded-wait settings of the tensor-core kernels: the device word in which a
@@ -92,8 +93,11 @@ int launch_embed(const BatchDesc& b, float* const* z, const void* w_in, const vo
                  const void* g = nullptr, void* xg = nullptr, float* ss = nullptr, int ss_ld = 0);
 int launch_rmsnorm(const float* x, const void* g, void* out, int rows, int d, float eps,
                    int dtype, cudaStream_t s);
+// rope3d: (t, y, x) positions over a raster of grid_w columns (else p0 + j)
 int launch_rope_table(const BatchDesc& b, float* cos_t, float* sin_t, int head_dim,
-                      double theta, cudaStream_t s);
+                      double theta, cudaStream_t s, bool rope3d = false, int grid_w = 1);
+// SwiGLU on an fp32 [rows][2F] projection in the interleaved gate/up layout -> out [rows][F]
+int launch_swiglu(const float* gu, void* out, int rows, int F, int dtype, cudaStream_t s);
 int launch_rope_scatter(const BatchDesc& b, const float* qkv, const float* cos_t,
                         const float* sin_t, void* q_out, void* k_layer, void* v_layer,
                         int n_heads, int head_dim, int dtype, cudaStream_t s);
@@ -106,7 +110,7 @@ int launch_exact_velocity_euler(float* z, const float* z0, float tau, float tau_
                                 cudaStream_t s);
 
 // GEMM C = A B^T, A [M][K], B [N][K] (both K-contiguous).
-enum Epilogue { EPI_F32 = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_STORE = 3, EPI_QKV = 4 };
+enum Epilogue { EPI_F32 = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_STORE = 3, EPI_QKV = 4, EPI_SWIGLU = 5 };
 int launch_gemm(const void* A, const void* B, void* C, int M, int N, int K, int epi, int dtype,
                 cudaStream_t s);
 

@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // fused RMSNorm of the A rows: 1 / rms of this row from the producer's partial sums
       float rinv = 1.f;
-      if ((EPI == EPI_QKV || EPI == EPI_GELU) && args.ss_in && live) {
+      if ((EPI == EPI_QKV || EPI == EPI_GELU || EPI == EPI_SWIGLU) && args.ss_in && live) {
         float ss = 0.f;
         for (int t2 = 0; t2 < args.ss_n; ++t2) ss += args.ss_in[(size_t)row * args.ss_ld + t2];
         rinv = rsqrtf(ss / (float)args.norm_d + args.norm_eps);
@@ -404,6 +404,26 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (cg == 0 && rr < args.M) args.ss_out[(size_t)rr * args.ss_ld + n0 / BN] = t;
           }
         }
+      } else if (EPI == EPI_SWIGLU) {
+        // columns 128 b + [0, 64) of the tile are gate units, 128 b + [64, 128) their up
+        // partners: out[(n0 + 128 b) / 2 + c] = silu(gate) * up, bf16
+        for (int b = 0; b < BN / 128; ++b) {
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t rg[32], ru[32];
+            tmem_ld32(tbase + b * 128 + hf * 32, rg);
+            tmem_ld32(tbase + b * 128 + 64 + hf * 32, ru);
+            tmem_wait_ld(rg);
+            reg_fence(ru);
+            if (!live) continue;
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float g = __uint_as_float(rg[i]) * rinv, u = __uint_as_float(ru[i]) * rinv;
+              v[i] = g / (1.f + __expf(-g)) * u;
+            }
+            store_bf16x32((__nv_bfloat16*)args.C + (size_t)row * args.ldc + (n0 + b * 128) / 2 + hf * 32, v);
+          }
+        }
       } else {
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
@@ -514,6 +534,7 @@ int gemm_tc_block_n(int M, int N, int hd, int epi, int sms, bool pair) {
   for (int bn : cands) {
     if (N % bn) continue;
     if (epi == EPI_QKV && (bn % 128 || hd % bn)) continue;
+    if (epi == EPI_SWIGLU && bn % 128) continue;   // whole gate / up block pairs
     const long long tiles = m_tiles * (N / bn);
     const long long cost = ((tiles + sms - 1) / sms) * (bn + 128);
     if (!best || cost < best_cost) {
@@ -563,6 +584,8 @@ int launch_gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& a
   SFM_GTC(128, EPI_RESID)
   SFM_GTC(128, EPI_STORE)
   SFM_GTC(128, EPI_QKV)
+  SFM_GTC(256, EPI_SWIGLU)
+  SFM_GTC(128, EPI_SWIGLU)
 #undef SFM_GTC
   return SFM_EINVAL;
 }

@@ -265,8 +265,12 @@ int launch_rmsnorm(const float* x, const void* g, void* out, int rows, int d, fl
 // ---------------------------------------------------------------------------
 // RoPE table: cos/sin [rows][D_h/2] for positions p0[sess] + j, in fp64.
 // ---------------------------------------------------------------------------
+// 3-D form (rope3d): pair i belongs to the time band (the first half - 2 ns pairs), the
+// row band or the column band (ns = head_dim / 6 pairs each); within a band of n_b pairs,
+// pair k turns by pos_axis * theta^(-k / n_b); positions (t_unit, y, x) for video token j
+// = y grid_w + x, (t_unit, 0, 0) for audio.
 __global__ void rope_table_kernel(BatchDesc b, float* __restrict__ cos_t, float* __restrict__ sin_t,
-                                  int half, double theta) {
+                                  int half, double theta, int rope3d, int grid_w) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   const int rows = b.n * b.n_tok;
   if (idx >= rows * half) return;
@@ -274,19 +278,69 @@ __global__ void rope_table_kernel(BatchDesc b, float* __restrict__ cos_t, float*
   const int i = idx - r * half;
   const int sess = r / b.n_tok;
   const int j = r - sess * b.n_tok;
-  const double pos = (double)(b.p0[sess] + j);
-  const double w = pow(theta, -2.0 * (double)i / (double)(2 * half));
+  double ang;
+  if (rope3d) {
+    const int ns = (2 * half) / 6, nt = half - 2 * ns;
+    const bool video = j < b.n_video;
+    double pos;
+    int k, nb;
+    if (i < nt) {
+      pos = (double)b.t_unit[sess];
+      k = i;
+      nb = nt;
+    } else if (i < nt + ns) {
+      pos = video ? (double)(j / grid_w) : 0.0;
+      k = i - nt;
+      nb = ns;
+    } else {
+      pos = video ? (double)(j % grid_w) : 0.0;
+      k = i - nt - ns;
+      nb = ns;
+    }
+    ang = pos * pow(theta, -(double)k / (double)nb);
+  } else {
+    const double pos = (double)(b.p0[sess] + j);
+    ang = pos * pow(theta, -2.0 * (double)i / (double)(2 * half));
+  }
   double sn, cs;
-  sincos(pos * w, &sn, &cs);
+  sincos(ang, &sn, &cs);
   cos_t[idx] = (float)cs;
   sin_t[idx] = (float)sn;
 }
 
 int launch_rope_table(const BatchDesc& b, float* cos_t, float* sin_t, int head_dim, double theta,
-                      cudaStream_t s) {
+                      cudaStream_t s, bool rope3d, int grid_w) {
   const int half = head_dim / 2;
   const int total = b.n * b.n_tok * half;
-  rope_table_kernel<<<(total + 255) / 256, 256, 0, s>>>(b, cos_t, sin_t, half, theta);
+  if (rope3d && grid_w < 1) return SFM_EINVAL;
+  rope_table_kernel<<<(total + 255) / 256, 256, 0, s>>>(b, cos_t, sin_t, half, theta,
+                                                        rope3d ? 1 : 0, grid_w);
+  return record_cuda(cudaGetLastError());
+}
+
+// SwiGLU of an fp32 projection in the interleaved layout: column 128 b + c (c < 64) is gate
+// unit 64 b + c and column 128 b + 64 + c its up partner; out = silu(gate) * up.
+template <typename T>
+__global__ void swiglu_kernel(const float* __restrict__ gu, T* __restrict__ out, long long n, int F) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n) return;
+  const long long r = idx / F;
+  const int f = (int)(idx - r * F);
+  const float* row = gu + r * 2 * (long long)F;
+  const int col = (f / 64) * 128 + (f % 64);
+  const float g = row[col], u = row[col + 64];
+  out[idx] = from_f<T>(g / (1.f + expf(-g)) * u);
+}
+
+int launch_swiglu(const float* gu, void* out, int rows, int F, int dtype, cudaStream_t s) {
+  const long long n = (long long)rows * F;
+  if (n == 0) return SFM_OK;
+  if (F % 64) return SFM_EUNSUPPORTED;
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  if (dtype == SFM_DTYPE_BF16)
+    swiglu_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(gu, (__nv_bfloat16*)out, n, F);
+  else
+    swiglu_kernel<float><<<blocks, 256, 0, s>>>(gu, (float*)out, n, F);
   return record_cuda(cudaGetLastError());
 }
 

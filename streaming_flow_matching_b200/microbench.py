@@ -198,10 +198,41 @@ def bench_guided(layers, cache_units, n_steps, scale, warmup, reps):
             "guided_steps_per_s": n_steps / ms_guided * 1e3}
 
 
+def bench_units(layers, cache_units, n_units, warmup, reps):
+    """A multi-unit pass (sfm_velocity_units) at the 640x368 unit: n_units units after a
+    cache_units-unit cache (0: a scene's first pass), all at tau = 0, 28 layers by default."""
+    w = S.V02.replace(name=f"v0.2-{layers}L", n_layers=layers, cache_units=max(cache_units, 1))
+    dev = torch.device("cuda", 0)
+    weights = S.make_weights(w, device=dev)
+    cap = max(cache_units + n_units, 1)
+    pool = cap * w.unit_kv_tokens + w.n_tokens
+    p = Performer.from_workload(w, weights, pool_tokens=pool, max_sessions=n_units)
+    s_id = p.open_session(cap)
+    if cache_units:
+        k, v = S.make_kv_slices(w, cache_units, device=dev)
+        p.kvcache_append(s_id, k, v)
+        del k, v
+    g = torch.Generator(device=dev)
+    g.manual_seed(61)
+    zs = [torch.randn(w.n_tokens, w.c_lat, generator=g, device=dev) for _ in range(n_units)]
+    vs = [torch.empty_like(z) for z in zs]
+    taus = [0.0] * n_units
+    ms = _time(lambda: p.velocity_units(s_id, zs, taus, v_outs=vs), warmup, reps)
+    p.check_device_error()
+    n = w.n_tokens
+    valid = cache_units * w.unit_kv_tokens
+    # visible keys: the cache plus the units up to each query's own
+    attn = sum(4 * n * (valid + (u + 1) * n) * w.hd for u in range(n_units))
+    gemm = n_units * (2 * n * w.d_model * 3 * w.hd + 2 * n * w.hd * w.d_model + 4 * n * w.d_model * w.d_mlp)
+    flop = layers * (attn + gemm)
+    return {"case": "units", "layers": layers, "units": n_units, "cache_tokens": valid,
+            "ms": ms, "tflops": flop / (ms / 1e3) / 1e12}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["attention", "append", "euler", "linear", "step", "guided",
-                                    "sweep"])
+                                    "units", "sweep"])
     ap.add_argument("--cache-units", type=int, default=4)
     ap.add_argument("--m", type=int, default=924)
     ap.add_argument("--k", type=int, default=3072)
@@ -233,6 +264,8 @@ def main():
         out.append(bench_step(a.layers, a.cache_units, a.warmup, a.reps))
     elif a.case == "guided":
         out.append(bench_guided(a.layers, a.cache_units, a.steps, a.scale, a.warmup, a.reps))
+    elif a.case == "units":
+        out.append(bench_units(a.layers, a.cache_units, a.units, a.warmup, a.reps))
     else:
         for m, n, k, e in [(924, 9216, 3072, "f32"), (924, 3072, 3072, "resid"),
                            (924, 12288, 3072, "gelu"), (924, 3072, 12288, "resid")]:

@@ -39,11 +39,13 @@ class Performer:
 
     def __init__(self, *, n_layers, d_model, n_heads, head_dim, d_mlp, c_lat, n_video, n_audio,
                  unit_kv_tokens, pool_tokens, max_sessions=1, dtype=torch.bfloat16, ring=True,
-                 rope_theta=10000.0, rms_eps=1e-6, weights=None):
+                 rope_theta=10000.0, rms_eps=1e-6, weights=None, mlp="gelu", rope="1d", grid_w=0):
         self.dtype = dtype
         self.cfg = L.sfm_config(n_layers, d_model, n_heads, head_dim, d_mlp, c_lat, n_video,
                                 n_audio, unit_kv_tokens, max_sessions, pool_tokens, _DT[dtype],
-                                int(ring), rope_theta, rms_eps)
+                                int(ring), rope_theta, rms_eps,
+                                {"gelu": L.SFM_MLP_GELU, "swiglu": L.SFM_MLP_SWIGLU}[mlp],
+                                {"1d": L.SFM_ROPE_1D, "3d": L.SFM_ROPE_3D}[rope], grid_w)
         self.n_tok = n_video + n_audio
         self.shape = dict(n_layers=n_layers, n_heads=n_heads, head_dim=head_dim, c_lat=c_lat)
         self._weights = weights           # keeps the borrowed device memory alive
@@ -63,7 +65,8 @@ class Performer:
                    n_audio=w.n_audio, unit_kv_tokens=w.unit_kv_tokens, pool_tokens=pool_tokens,
                    max_sessions=max_sessions,
                    dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32, ring=ring,
-                   rope_theta=w.rope_theta, rms_eps=w.rms_eps, weights=weights)
+                   rope_theta=w.rope_theta, rms_eps=w.rms_eps, weights=weights, mlp=w.mlp,
+                   rope=w.rope, grid_w=w.grid_w)
 
     def _weights_struct(self, w):
         n = self.cfg.n_layers

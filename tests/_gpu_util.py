@@ -17,7 +17,8 @@ WIDE_BF16 = S.Workload("wide-bf16", 1, 4224, 2, 128, 256, 16, 24, 4, 32, 3, 2, "
 
 def ocfg(w):
     return O.Config(w.n_layers, w.d_model, w.n_heads, w.head_dim, w.d_mlp, w.c_lat, w.n_video,
-                    w.n_audio, w.unit_kv_tokens, w.rope_theta, w.rms_eps)
+                    w.n_audio, w.unit_kv_tokens, w.rope_theta, w.rms_eps, mlp=w.mlp,
+                    rope_mode=w.rope, grid_w=w.grid_w)
 
 
 def rel_l2(got, ref):

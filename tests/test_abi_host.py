@@ -36,7 +36,8 @@ def test_every_declared_symbol_is_exported():
 def cfg(**kw):
     base = dict(n_layers=2, d_model=256, n_heads=4, head_dim=64, d_mlp=1024, c_lat=16,
                 n_video=64, n_audio=4, unit_kv_tokens=96, max_sessions=1, pool_tokens=0,
-                dtype=L.SFM_DTYPE_FP32, ring=1, rope_theta=1e4, rms_eps=1e-6)
+                dtype=L.SFM_DTYPE_FP32, ring=1, rope_theta=1e4, rms_eps=1e-6, mlp=0, rope=0,
+                grid_w=0)
     base.update(kw)
     return L.sfm_config(*[base[f] for f, _ in L.sfm_config._fields_])
 
@@ -53,6 +54,10 @@ def cfg(**kw):
     (dict(dtype=L.SFM_DTYPE_BF16), L.SFM_EUNSUPPORTED),          # bf16 needs D_h = 128
     (dict(dtype=L.SFM_DTYPE_BF16, head_dim=128, n_heads=2, d_model=192), L.SFM_EUNSUPPORTED),
     (dict(head_dim=48), L.SFM_EUNSUPPORTED),
+    (dict(mlp=2), L.SFM_EINVAL),
+    (dict(rope=2), L.SFM_EINVAL),
+    (dict(rope=1, grid_w=0), L.SFM_EINVAL),                   # 3-D RoPE needs the raster width
+    (dict(mlp=1, d_mlp=1000), L.SFM_EUNSUPPORTED),           # SwiGLU blocks of 64 units
 ])
 def test_create_rejects_bad_config_on_host(bad, code):
     h = C.c_void_p()

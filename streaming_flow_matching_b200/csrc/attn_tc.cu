@@ -17,12 +17,14 @@
 //               (P_t aliases S_t in TMEM).
 //   warps 2-5   softmax of tile A, warps 6-9 softmax of tile B (thread = query
 //               row): one pass over the S row in TMEM computes
-//               p = 2^(s scale - m) against the running max m together with the
-//               tile's max; P is held in registers and written back over S as
-//               packed bf16.  Only when a row's max grows by more than 2^8
-//               (decided per warp: the TMEM accesses are collective) is O
-//               rescaled in TMEM and P recomputed from S.  Final O / l written
-//               as bf16 (one split) or as fp32 partials + log2-sum-exp.
+//               p = 2^(s scale - m) against the running max m; P is held in
+//               registers and written back over S as packed bf16.  A row's max
+//               can only have grown by more than 2^8 if its tile sum of p passed
+//               2^8, so only then is the tile's exact max taken (a second pass
+//               over S), and only when it did grow by more (decided per warp: the
+//               TMEM accesses are collective) is O rescaled in TMEM and P
+//               recomputed from S.  Final O / l written as bf16 (one split) or as
+//               fp32 partials + log2-sum-exp.
 // TMEM columns: tile A S/P [0,128) O [128,256); tile B S/P [256,384) O [384,512).
 // The last, partial key tile is masked in S, and its V rows past the key range
 // are zeroed in shared memory before P V, so rows outside the range never
@@ -310,11 +312,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_st_wait();
       }
       // P = 2^(s scale - m) with m the running row max.  From the second key tile on, one
-      // pass over the S row computes P against the running max and the tile's max
-      // together; only when some row of the warp grows by more than 2^8 is that
-      // attempt dropped: O is rescaled and P recomputed from S (still intact in TMEM,
-      // as P is held in registers until the row is done).  The first tile takes its
-      // max first.  Loads of the next 32-column chunk overlap work on the current one.
+      // pass over the S row computes P against the running max; the row's tile sum of P
+      // bounds its growth (some p > 2^8 only if the sum passed 2^8), so the tile's exact
+      // max is taken only then, and only when some row of the warp grows by more than
+      // 2^8 is the attempt dropped: O is rescaled and P recomputed from S (still intact
+      // in TMEM, as P is held in registers until the row is done).  The first tile takes
+      // its max first.  Loads of the next 32-column chunk overlap work on the current one.
       uint32_t pk[4][16];
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
       float mx = -INFINITY;
@@ -323,7 +326,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         // a row with no visible key so far (block-causal, a later split) has m = -inf:
         // its attempt below is dropped by the rescale test, so any finite base serves
         const float neg_m = m == -INFINITY ? 0.f : -m;
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         uint32_t u[2][32];
         tmem_ld32(tmem + lane_base + col_s, u[0]);
         tmem_wait_ld(u[0]);
@@ -333,7 +335,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           const float* sv = reinterpret_cast<const float*>(u[c & 1]);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            m4[i & 3] = fmax3(m4[i & 3], sv[2 * i], sv[2 * i + 1]);
             const float p0 = ex2_approx(fmaf(sv[2 * i], sc, neg_m));
             const float p1 = ex2_approx(fmaf(sv[2 * i + 1], sc, neg_m));
             l4[(2 * i) & 3] += p0;
@@ -342,8 +343,30 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           if (c + 1 < 4) tmem_wait_ld(u[(c + 1) & 1]);
         }
-        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
-        if (__any_sync(0xffffffffu, mx > m + kRescaleLog2)) {
+        // a row's max can only have grown by more than 2^8 if its tile sum of p passed 2^8
+        // (every p > 0); only then is the tile's exact row max taken, from S (intact in TMEM)
+        const float lt = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        bool grown = false;
+        if (__any_sync(0xffffffffu, !(lt <= 256.f))) {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t w[32];
+            tmem_ld32(tmem + lane_base + col_s + c * 32, w);
+            tmem_wait_ld(w);
+            const float* sv = reinterpret_cast<const float*>(w);
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              m4[0] = fmax3(m4[0], sv[i], sv[i + 1]);
+              m4[1] = fmax3(m4[1], sv[i + 2], sv[i + 3]);
+              m4[2] = fmax3(m4[2], sv[i + 4], sv[i + 5]);
+              m4[3] = fmax3(m4[3], sv[i + 6], sv[i + 7]);
+            }
+          }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sc;
+          grown = __any_sync(0xffffffffu, mx > m + kRescaleLog2);
+        }
+        if (grown) {
           // O_t's previous P V has completed (S_t(j) was issued after it): rescale it
           const float m_new = fmaxf(m, mx);
           const float alpha = m == -INFINITY ? 0.f : ex2_approx(m - m_new);   // O, l are 0 then

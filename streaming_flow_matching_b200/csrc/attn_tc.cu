@@ -287,14 +287,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = true;
     const float sc = args.scale_log2;
     for (int j = 0; j < T && ok; ++j) {
+      // the key limits of this tile do not depend on S: settled before waiting for it
+      const int kvalid = nkeys - (t0 + j) * BKV;         // > 0; < BKV only on the last tile
+      const int kmine = my_keys - (t0 + j) * BKV;        // this row's; may be <= 0
+      const int kwarp = __reduce_min_sync(0xffffffffu, kmine);
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], (uint32_t)(j & 1), abort, args.err, 0x207, args.wait_ns))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int kvalid = nkeys - (t0 + j) * BKV;         // > 0; < BKV only on the last tile
-      const int kmine = my_keys - (t0 + j) * BKV;        // this row's; may be <= 0
-      const int kwarp = __reduce_min_sync(0xffffffffu, kmine);
       if (kwarp < BKV) {
         // partial tile for some row of the warp: overwrite the row's logits past its
         // key limit with -inf (the TMEM accesses are warp-collective)

@@ -485,6 +485,20 @@ typedef struct sfm_plan {
   int fused_norm;
 } sfm_plan;
 SFM_API int sfm_get_plan(const sfm_handle* h, sfm_plan* out);
+
+/*
+ * The key-range split counts the tcgen05 attention of a batched f_theta call
+ * uses (introspection, no counterpart in the method).  n_sessions sessions of
+ * rows_per_session query rows each, session i attending to n_keys[i] keys (its
+ * cached tokens plus the current unit), n_heads heads, on a device of sms SMs:
+ * splits[i] (host memory, n_sessions entries, caller-owned) receives session i's
+ * count in [1, 16].  A session of one split has its output written by the
+ * attention kernel itself; the others' partial results are merged.  Host only
+ * (no device work).  SFM_EINVAL if a pointer is NULL, n_sessions is outside
+ * [1, 16], or rows_per_session, n_heads, sms or an n_keys[i] is < 1.
+ */
+SFM_API int sfm_attention_batch_splits(int n_sessions, int rows_per_session, const long long* n_keys,
+                                       int n_heads, int sms, int* splits);
 SFM_API const char* sfm_strerror(int status);
 /* The cudaError_t of the last failed CUDA call made by this library on this
  * host thread (0 if none). */

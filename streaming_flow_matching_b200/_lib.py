@@ -93,6 +93,7 @@ def _load():
         "sfm_check_call_error": (i, [C.POINTER(i)]),
         "sfm_test_fault": (i, [vp, i, ll]),
         "sfm_get_plan": (i, [vp, C.POINTER(sfm_plan)]),
+        "sfm_attention_batch_splits": (i, [i, i, C.POINTER(ll), i, i, C.POINTER(i)]),
         "sfm_euler_update": (i, [vp, vp, f, ll, vp]),
         "sfm_fm_solve_exact_velocity": (i, [vp, vp, vp, C.POINTER(f), i, vp]),
         "sfm_profile_begin": (i, [i]),
@@ -121,10 +122,21 @@ EXPORTS = ["sfm_create", "sfm_destroy", "sfm_session_open", "sfm_session_reset",
            "sfm_attention_noalloc", "sfm_linear", "sfm_euler_update", "sfm_fm_solve_exact_velocity",
            "sfm_profile_begin", "sfm_profile_end", "sfm_kernel_launch_count",
            "sfm_check_device_error", "sfm_clear_device_error", "sfm_check_call_error",
-           "sfm_test_fault", "sfm_get_plan", "sfm_strerror", "sfm_last_cuda_error"]
+           "sfm_test_fault", "sfm_get_plan", "sfm_attention_batch_splits", "sfm_strerror",
+           "sfm_last_cuda_error"]
 
 PROF_KINDS = ["append", "attention", "attention_merge", "gemm_qkv", "gemm_o", "gemm_up",
               "gemm_down", "rowops", "head_euler"]
+
+
+def attention_batch_splits(rows_per_session, n_keys, n_heads, sms=148):
+    """The split counts the batched attention gives each session (host only)."""
+    n = len(n_keys)
+    keys = (C.c_longlong * max(1, n))(*n_keys)
+    out = (C.c_int * max(1, n))()
+    check(lib.sfm_attention_batch_splits(n, rows_per_session, keys, n_heads, sms, out),
+          "sfm_attention_batch_splits")
+    return list(out[:n])
 
 
 def profile_begin(max_launches=1 << 16):

@@ -1,6 +1,7 @@
 // C ABI of libsfm: argument validation, ownership of the K/V pool and the
 // scratch activations, session bookkeeping, and the per-step launch sequence
 // of f_theta.  Every error is caught on the host before any launch.
+#include <limits.h>
 #include <math.h>
 #include <string.h>
 
@@ -262,7 +263,8 @@ int run_step(sfm_handle* h, const BatchDesc& b, const AttnDesc& ad, float* const
     ss_n = d / bn;
     return g;
   };
-  const int splits = tc ? attention_tc_splits_batch(ad, c.n_heads, h->sms) : 1;
+  int splits[kMaxBatch];   // key splits of each session's attention
+  if (tc) attention_tc_splits_batch(ad, c.n_heads, h->sms, splits);
   for (int l = 0; l < c.n_layers; ++l) {
     if (!tc) {
       ProfScope ps(SFM_PROF_ROWOPS, s);
@@ -296,7 +298,7 @@ int run_step(sfm_handle* h, const BatchDesc& b, const AttnDesc& ad, float* const
                                   h->o_part, h->lse_part, h->gd, s));
     } else {
       SFM_TRY(launch_attention(ad, h->q, h->layer_k(l), h->layer_v(l), h->ao, c.n_heads,
-                               c.head_dim, dt, splits, h->o_part, h->lse_part, s));
+                               c.head_dim, dt, 1, h->o_part, h->lse_part, s));
     }
     {
       ProfScope ps(SFM_PROF_GEMM_O, s);
@@ -1117,6 +1119,22 @@ int sfm_get_plan(const sfm_handle* h, sfm_plan* out) {
     out->k_splits[i] = ks[i];
   }
   out->fused_norm = h->has_weights && h->cfg.dtype == SFM_DTYPE_BF16 ? 1 : 0;
+  return SFM_OK;
+}
+
+int sfm_attention_batch_splits(int n_sessions, int rows_per_session, const long long* n_keys,
+                               int n_heads, int sms, int* splits) {
+  if (!n_keys || !splits || n_sessions < 1 || n_sessions > kMaxBatch || rows_per_session < 1 ||
+      n_heads < 1 || sms < 1)
+    return SFM_EINVAL;
+  AttnDesc a{};
+  a.n = n_sessions;
+  a.rows_per = rows_per_session;
+  for (int i = 0; i < n_sessions; ++i) {
+    if (n_keys[i] < 1 || n_keys[i] > INT_MAX) return SFM_EINVAL;
+    a.nkeys[i] = (int)n_keys[i];
+  }
+  attention_tc_splits_batch(a, n_heads, sms, splits);
   return SFM_OK;
 }
 

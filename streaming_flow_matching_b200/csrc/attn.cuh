@@ -39,19 +39,35 @@ int launch_attention(const AttnDesc& a, const void* q, const void* k, const void
                      int n_heads, int head_dim, int dtype, int n_splits, float* o_part,
                      float* lse_part, cudaStream_t s);
 
+// The sessions one merge launch combines, all of the same split count: session
+// sess[k] (k < n) owns rows [sess[k] * rows_per, (sess[k] + 1) * rows_per).
+struct MergeDesc {
+  int rows_per;
+  int n;
+  int sess[kMaxBatch];
+};
 int launch_attention_merge(const float* o_part, const float* lse_part, void* o,
-                           long long total_rows, int n_heads, int n_splits, cudaStream_t s);
+                           long long total_rows, int n_heads, int n_splits, const MergeDesc& md,
+                           cudaStream_t s);
 
 // tcgen05 attention (bf16, D = 128).  Split count for a batch; the SM count is an input so the choice is
 // reproducible (the standalone call assumes 148).
 // unit_rows > 0: block-causal (see AttnDesc), which shortens the early query blocks.
 int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys, int n_heads,
                         int sms, int unit_rows = 0);
-// A batch whose sessions have their own key counts (AttnDesc::nkeys).
-int attention_tc_splits_batch(const AttnDesc& a, int n_heads, int sms);
+// A batch whose sessions have their own key counts (AttnDesc::nkeys): one split
+// count per session into ns[0 .. a.n); returns the largest.
+int attention_tc_splits_batch(const AttnDesc& a, int n_heads, int sms, int* ns);
 // mq: map over the query rows [rows][H][128]; mk, mv: maps over the key rows, of
 // which this call uses rows kv_row0 + kbase[s] + [0, nkeys[s]).
 // gd: error word, wait bound and test-only fault of the launch.
+// ns: the split count of each session (1..kMaxSplits); sessions of more than one
+// split write fp32 partials to o_part / lse_part ([split][rows][H][D], [split][rows][H])
+// that a merge then combines into o.
+int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const AttnDesc& a, int kv_row0, int n_heads, const int* ns, void* o,
+                        float* o_part, float* lse_part, const Guard& gd, cudaStream_t s);
+// every session split n_splits ways
 int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const AttnDesc& a, int kv_row0, int n_heads, int n_splits, void* o,
                         float* o_part, float* lse_part, const Guard& gd, cudaStream_t s);

@@ -57,16 +57,20 @@ __global__ void attn_f32_kernel(AttnDesc a, const float* __restrict__ q,
 // of a row are in flight together.  The split count is a template parameter so a
 // thread holds exactly its splits' values (a fixed 16-slot version needed 94
 // registers and ran at a quarter of the warps an SM can hold).
+// The rows of the sessions md lists, each of S partials (one launch per split count).
 template <int S>
 __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict__ o_part,
                                                          const float* __restrict__ lse_part,
                                                          __nv_bfloat16* __restrict__ o,
-                                                         long long total_rows, int H) {
-  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+                                                         long long total_rows, int H, MergeDesc md) {
+  const unsigned gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (gw >= total_rows * H) return;
-  const long long row = gw / H;
-  const int h = (int)(gw - row * H);
+  const unsigned per = (unsigned)md.rows_per * (unsigned)H;   // (row, head) pairs of a session
+  if (gw >= (unsigned)md.n * per) return;
+  const unsigned k = gw / per, rh = gw - k * per;
+  const unsigned r = rh / (unsigned)H;
+  const int h = (int)(rh - r * (unsigned)H);
+  const long long row = (long long)md.sess[k] * md.rows_per + r;
   const long long ld = (long long)H * 128;
   float lse[S];
   float4 p[S];
@@ -99,15 +103,15 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
 
 template <int S>
 static void launch_merge_s(const float* o_part, const float* lse_part, void* o, long long total_rows,
-                           int n_heads, int n_splits, cudaStream_t s) {
+                           int n_heads, int n_splits, const MergeDesc& md, cudaStream_t s) {
   if constexpr (S > 1) {
     if (n_splits != S) {
-      launch_merge_s<S - 1>(o_part, lse_part, o, total_rows, n_heads, n_splits, s);
+      launch_merge_s<S - 1>(o_part, lse_part, o, total_rows, n_heads, n_splits, md, s);
       return;
     }
-    const long long warps = total_rows * n_heads;
+    const long long warps = (long long)md.n * md.rows_per * n_heads;
     attn_merge_kernel<S><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, s>>>(
-        o_part, lse_part, (__nv_bfloat16*)o, total_rows, n_heads);
+        o_part, lse_part, (__nv_bfloat16*)o, total_rows, n_heads, md);
   }
 }
 
@@ -137,9 +141,12 @@ int launch_attention(const AttnDesc& a, const void* q, const void* k, const void
 }
 
 int launch_attention_merge(const float* o_part, const float* lse_part, void* o,
-                           long long total_rows, int n_heads, int n_splits, cudaStream_t s) {
-  if (n_splits < 2 || n_splits > kMaxSplits) return SFM_EINVAL;
-  launch_merge_s<kMaxSplits>(o_part, lse_part, o, total_rows, n_heads, n_splits, s);
+                           long long total_rows, int n_heads, int n_splits, const MergeDesc& md,
+                           cudaStream_t s) {
+  if (n_splits < 2 || n_splits > kMaxSplits || md.rows_per < 1 || md.n < 1 || md.n > kMaxBatch ||
+      (long long)md.n * md.rows_per * n_heads * 32 >= (1LL << 31))
+    return SFM_EINVAL;
+  launch_merge_s<kMaxSplits>(o_part, lse_part, o, total_rows, n_heads, n_splits, md, s);
   return record_cuda(cudaGetLastError());
 }
 

@@ -6,7 +6,11 @@
 // range per session, D = 128.
 //
 // One CTA = one (session, head, 256-query block, key split): two 128-row
-// query tiles A and B share every K/V tile.  320 threads:
+// query tiles A and B share every K/V tile.  Each session has its own split
+// count; the CTAs are numbered session by session in a host-given order (longest
+// CTAs first, so the SMs finish together), and within a session split, head,
+// query block, the query block fastest: the CTAs that read the same K/V tiles
+// start together.  320 threads:
 //   warp 0      TMA producer: both Q tiles once; K tiles (128 keys x 128 dims)
 //               in a 3-stage ring, V tiles in a 2-stage ring (128-byte swizzle)
 //   warp 1      TMEM allocator; lane 0 issues tcgen05.mma, alternating tiles:
@@ -38,6 +42,9 @@
 // it weight 0.
 #include <math.h>
 
+#include <algorithm>
+#include <vector>
+
 #include "attn.cuh"
 #include "sm100.cuh"
 
@@ -65,14 +72,15 @@ constexpr float kRescaleLog2 = 8.0f;
 struct Args {
   AttnDesc a;
   int H;
-  int n_splits;
+  int ns[kMaxBatch];           // key splits of each session (1: O written directly)
+  int order[kMaxBatch];        // sessions in CTA order
   int qtiles;                  // 256-row query blocks per session
   float scale_log2;
   long long total_rows;
   int kv_row0;                 // row offset of this layer inside the K/V tensor maps
   __nv_bfloat16* o;            // [total_rows][H][D] (one split)
-  float* o_part;               // [n_splits][total_rows][H][D]
-  float* lse_part;             // [n_splits][total_rows][H]
+  float* o_part;               // [split][total_rows][H][D] (sessions of more than one split)
+  float* lse_part;             // [split][total_rows][H]
   int* err;
   unsigned long long wait_ns;  // bound of every wait
   int fault;                   // SFM_FAULT_ATTN_NO_LOADS: the producer issues no loads (test only)
@@ -99,11 +107,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* drain = o_done + QT;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // the CTA's work, decoded once below: the softmax warps read it back from shared
+  // memory where they need it, so that none of it holds registers through their key loop
+  volatile int* cta_info = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sess = blockIdx.x / args.qtiles;
-  const int qb = blockIdx.x - sess * args.qtiles;
-  const int h = blockIdx.y, split = blockIdx.z;
+  int rem = blockIdx.x, sess = args.order[0];
+  for (int i = 0; i < args.a.n; ++i) {
+    sess = args.order[i];
+    const int c = args.ns[sess] * args.H * args.qtiles;
+    if (rem < c) break;
+    rem -= c;
+  }
+  const int n_splits = args.ns[sess];
+  const int qb = rem % args.qtiles;
+  rem /= args.qtiles;
+  const int h = rem % args.H, split = rem / args.H;
   const long long row0 = (long long)sess * args.a.rows_per + (long long)qb * ROWS;
   // keys of this CTA: up to the limit of its last query row (block-causal: the
   // rows' own limits are masked per row below)
@@ -111,7 +130,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int nkeys = attn_key_limit(args.a.nkeys[sess], args.a.rows_per, args.a.unit_rows, q_last);
   const long long kbase = args.a.kbase[sess];
   const int ntiles = (nkeys + BKV - 1) / BKV;
-  const int tps = (ntiles + args.n_splits - 1) / args.n_splits;
+  const int tps = (ntiles + n_splits - 1) / n_splits;
   const int t0 = min(ntiles, split * tps);
   const int t1 = min(ntiles, t0 + tps);
   const int T = t1 - t0;
@@ -133,6 +152,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(drain, 1);
     *abort = 0;
+    cta_info[0] = h;
+    cta_info[1] = split;
+    cta_info[2] = n_splits;
+    cta_info[3] = sess;
+    cta_info[4] = qb;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -460,7 +484,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&o_done[t], (uint32_t)((T - 1) & 1), abort, args.err, 0x20A, args.wait_ns))) ok = false;
       tc_fence_after();
     }
-    const long long grow = row0 + t * BQ + r;
+    const int h_o = cta_info[0], split_o = cta_info[1], n_splits_o = cta_info[2];
+    const long long row0_o = (long long)cta_info[3] * args.a.rows_per + (long long)cta_info[4] * ROWS;
+    const long long grow = row0_o + t * BQ + r;
     const long long ld = (long long)args.H * D;
     const bool have = ok && T > 0 && l > 0.f;
     const float inv = have ? 1.f / l : 0.f;
@@ -493,36 +519,36 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       __syncwarp();
-      const long long grow0 = row0 + t * BQ + quarter * 32;   // global row of the warp's lane 0
+      const long long grow0 = row0_o + t * BQ + quarter * 32;   // global row of the warp's lane 0
       for (int rr = 0; rr < 32; ++rr) {
         if (quarter * 32 + rr >= q_rows) break;               // warp-uniform
         const float4 f = stage[rr * 32 + (lane ^ rr)];        // columns 4 lane .. 4 lane + 3
-        if (args.n_splits == 1) {
+        if (n_splits_o == 1) {
           uint2 b;
           b.x = pack_bf16x2(f.x, f.y);
           b.y = pack_bf16x2(f.z, f.w);
-          *reinterpret_cast<uint2*>(args.o + (grow0 + rr) * ld + h * D + 4 * lane) = b;
+          *reinterpret_cast<uint2*>(args.o + (grow0 + rr) * ld + h_o * D + 4 * lane) = b;
         } else {
-          *reinterpret_cast<float4*>(args.o_part + ((long long)split * args.total_rows + grow0 + rr) * ld +
-                                     h * D + 4 * lane) = f;
+          *reinterpret_cast<float4*>(args.o_part + ((long long)split_o * args.total_rows + grow0 + rr) * ld +
+                                     h_o * D + 4 * lane) = f;
         }
       }
     } else if (r < q_rows) {
       // unwinding after a timed-out wait (loads may still land in shared memory):
       // zeros, written directly
       for (int c = 0; c < 4; ++c) {
-        if (args.n_splits == 1) {
-          uint4* d = reinterpret_cast<uint4*>(args.o + grow * ld + h * D + c * 32);
+        if (n_splits_o == 1) {
+          uint4* d = reinterpret_cast<uint4*>(args.o + grow * ld + h_o * D + c * 32);
           for (int q = 0; q < 4; ++q) d[q] = make_uint4(0u, 0u, 0u, 0u);
         } else {
-          float4* d = reinterpret_cast<float4*>(args.o_part + ((long long)split * args.total_rows + grow) * ld +
-                                                h * D + c * 32);
+          float4* d = reinterpret_cast<float4*>(args.o_part + ((long long)split_o * args.total_rows + grow) * ld +
+                                                h_o * D + c * 32);
           for (int q = 0; q < 8; ++q) d[q] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
     }
-    if (r < q_rows && args.n_splits > 1)
-      args.lse_part[((long long)split * args.total_rows + grow) * args.H + h] =
+    if (r < q_rows && n_splits_o > 1)
+      args.lse_part[((long long)split_o * args.total_rows + grow) * args.H + h_o] =
           have ? m + log2f(l) : -INFINITY;
   }
 
@@ -536,13 +562,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace atc
 
-// Split count from a cost model of the kernel, in microseconds on a B200:
+// Split counts from a cost model of the kernel, in microseconds on a B200:
 //   CTA time  = (key tiles of the CTA) x kStepUs + kCtaUs (set-up, output, hand-over),
-//   kernel    = max(waves x mean CTA time, longest CTA time), waves = ceil(CTAs / SMs),
 //   merge     = its bytes (fp32 partials of every split read, bf16 O written) / kMergeBps.
 // More splits fill the SMs and shorten the longest CTA; each split adds fixed cost and
 // merge traffic.  Block-causal calls count each query block's own key tiles.
 namespace {
+
+constexpr double kStepUs = 2.0, kCtaUs = 5.0, kMergeBps = 4.0e6;   // bytes per microsecond
 
 // key tiles of query block b of a session with `keys` keys
 long long block_tiles(int rows_per, long long keys, int unit_rows, int b) {
@@ -553,16 +580,15 @@ long long block_tiles(int rows_per, long long keys, int unit_rows, int b) {
   return (lim + atc::BKV - 1) / atc::BKV;
 }
 
-// Split count from a cost model of the kernel, in microseconds on a B200:
-//   CTA time  = (key tiles of the CTA) x kStepUs + kCtaUs (set-up, output, hand-over),
-//   kernel    = max(waves x mean CTA time, longest CTA time), waves = ceil(CTAs / SMs),
-//   merge     = its bytes (fp32 partials of every split read, bf16 O written) / kMergeBps.
-// More splits fill the SMs and shorten the longest CTA; each split adds fixed cost and
-// merge traffic.  tiles_of(i): key tiles of query block i (i < n_blocks); every block
-// runs n_heads CTAs per split; merge_rows = query rows x heads.
+double merge_us(double rows_heads, int s) {
+  return s > 1 ? (s * rows_heads * (atc::D + 1) * 4.0 + rows_heads * atc::D * 2.0) / kMergeBps : 0.0;
+}
+
+// One split count for identical sessions: kernel = max(waves x mean CTA time, longest
+// CTA time), waves = ceil(CTAs / SMs).  tiles_of(i): key tiles of query block i
+// (i < n_blocks); every block runs n_heads CTAs per split; merge_rows = query rows x heads.
 template <typename F>
 int choose_splits(F tiles_of, int n_blocks, int n_heads, double merge_rows, int sms) {
-  constexpr double kStepUs = 2.0, kCtaUs = 5.0, kMergeBps = 4.0e6;   // bytes per microsecond
   long long max_tiles = 0;
   for (int i = 0; i < n_blocks; ++i) max_tiles = tiles_of(i) > max_tiles ? tiles_of(i) : max_tiles;
   const long long ctas = (long long)n_blocks * n_heads;
@@ -580,13 +606,67 @@ int choose_splits(F tiles_of, int n_blocks, int n_heads, double merge_rows, int 
     const double waves = (double)((work + sms - 1) / sms);
     double us = waves * sum_t / n_blocks;
     if (max_t > us) us = max_t;
-    if (s > 1) us += (s * merge_rows * (atc::D + 1) * 4.0 + merge_rows * atc::D * 2.0) / kMergeBps;
+    us += merge_us(merge_rows, s);
     if (s == 1 || us < best_us) {
       best = s;
       best_us = us;
     }
   }
   return best;
+}
+
+// key tiles of CTA (split z of ns, query block b) of session i
+long long cta_tiles(const AttnDesc& a, int i, int b, int ns, int z) {
+  const long long t = block_tiles(a.rows_per, a.nkeys[i], a.unit_rows, b);
+  const long long tps = (t + ns - 1) / ns;
+  const long long t0 = z * tps < t ? z * tps : t;
+  return (t0 + tps < t ? t0 + tps : t) - t0;
+}
+
+// The kernel's CTA order: sessions by the key tiles of their longest CTA, longest
+// first (ties by index); within a session split, head, query block.
+void cta_order(const AttnDesc& a, const int* ns, int* order) {
+  const int qtiles = (a.rows_per + atc::ROWS - 1) / atc::ROWS;
+  long long len[kMaxBatch];
+  for (int i = 0; i < a.n; ++i) {
+    len[i] = cta_tiles(a, i, qtiles - 1, ns[i], 0);   // the last block sees the most keys
+    order[i] = i;
+  }
+  std::stable_sort(order, order + a.n, [&](int x, int y) { return len[x] > len[y]; });
+}
+
+// Kernel time of a per-session plan: its CTAs, in the kernel's order, each given to
+// the SM that frees first (a binary min-heap of the SMs' finishing times).
+double schedule_us(const AttnDesc& a, const int* ns, int n_heads, int sms, std::vector<double>& heap) {
+  const int qtiles = (a.rows_per + atc::ROWS - 1) / atc::ROWS;
+  int order[kMaxBatch];
+  cta_order(a, ns, order);
+  heap.assign((size_t)sms, 0.0);
+  std::vector<double> len((size_t)qtiles);
+  for (int k = 0; k < a.n; ++k) {
+    const int i = order[k];
+    for (int z = 0; z < ns[i]; ++z) {
+      for (int b = 0; b < qtiles; ++b) len[b] = (double)cta_tiles(a, i, b, ns[i], z) * kStepUs + kCtaUs;
+      for (int hh = 0; hh < n_heads; ++hh)
+        for (int b = 0; b < qtiles; ++b) {
+          // replace the root (earliest free SM) by its new finishing time and sift down
+          const double v = heap[0] + len[b];
+          size_t p = 0;
+          for (;;) {
+            size_t c = 2 * p + 1;
+            if (c >= heap.size()) break;
+            if (c + 1 < heap.size() && heap[c + 1] < heap[c]) ++c;
+            if (heap[c] >= v) break;
+            heap[p] = heap[c];
+            p = c;
+          }
+          heap[p] = v;
+        }
+    }
+  }
+  double mk = 0.0;
+  for (double t : heap) mk = t > mk ? t : mk;
+  return mk;
 }
 
 }  // namespace
@@ -601,25 +681,107 @@ int attention_tc_splits(int rows_per_session, int n_sessions, long long max_keys
       n_sessions * qtiles, n_heads, (double)n_sessions * rows_per_session * n_heads, sms);
 }
 
-// A batch whose sessions have their own key counts (ragged caches).
-int attention_tc_splits_batch(const AttnDesc& a, int n_heads, int sms) {
+// A batch whose sessions have their own key counts (ragged caches): a split count
+// per session.  Candidates: one count for every session (1..kMaxSplits), and
+// ns_i = ceil(T_i / L) (T_i: the tiles of session i's longest query block) for each
+// CTA length L at which some session's count changes.  Each candidate is scored by
+// list-scheduling its CTAs in the kernel's order (schedule_us) plus its merge; one
+// whose lower bound -- max(total CTA time / SMs, longest CTA) + merge -- cannot beat
+// the best scored so far is not scheduled.  A single session keeps the
+// identical-sessions model.
+int attention_tc_splits_batch(const AttnDesc& a, int n_heads, int sms, int* ns) {
   const int qtiles = (a.rows_per + atc::ROWS - 1) / atc::ROWS;
-  return choose_splits(
-      [&](int i) { return block_tiles(a.rows_per, a.nkeys[i / qtiles], a.unit_rows, i % qtiles); },
-      a.n * qtiles, n_heads, (double)a.n * a.rows_per * n_heads, sms);
+  if (a.n <= 1) {
+    ns[0] = a.n == 1 ? attention_tc_splits(a.rows_per, 1, a.nkeys[0], n_heads, sms, a.unit_rows) : 1;
+    return ns[0];
+  }
+  long long tmax[kMaxBatch], top = 0;
+  for (int i = 0; i < a.n; ++i) {
+    tmax[i] = block_tiles(a.rows_per, a.nkeys[i], a.unit_rows, qtiles - 1);
+    top = tmax[i] > top ? tmax[i] : top;
+  }
+  struct Cand {
+    int ns[kMaxBatch];
+    double lb;
+  };
+  std::vector<Cand> cands;
+  auto add = [&](const int* v) {
+    for (const Cand& c : cands)
+      if (std::equal(v, v + a.n, c.ns)) return;
+    Cand c{};
+    std::copy(v, v + a.n, c.ns);
+    double total = 0.0, longest = 0.0, merge = 0.0;
+    for (int i = 0; i < a.n; ++i) {
+      for (int z = 0; z < v[i]; ++z)
+        for (int b = 0; b < qtiles; ++b) {
+          const double t = (double)cta_tiles(a, i, b, v[i], z) * kStepUs + kCtaUs;
+          total += t * n_heads;
+          longest = t > longest ? t : longest;
+        }
+      merge += merge_us((double)a.rows_per * n_heads, v[i]);
+    }
+    c.lb = (total / sms > longest ? total / sms : longest) + merge;
+    cands.push_back(c);
+  };
+  int v[kMaxBatch];
+  for (int s = 1; s <= kMaxSplits; ++s) {
+    if (s > 1 && top / s < 2) break;
+    for (int i = 0; i < a.n; ++i) v[i] = s;
+    add(v);
+  }
+  std::vector<long long> lens;
+  for (int i = 0; i < a.n; ++i)
+    for (int s = 1; s <= kMaxSplits; ++s) lens.push_back((tmax[i] + s - 1) / s);
+  std::sort(lens.begin(), lens.end());
+  lens.erase(std::unique(lens.begin(), lens.end()), lens.end());
+  for (long long L : lens) {
+    if (L < 2) continue;
+    for (int i = 0; i < a.n; ++i) {
+      const long long s = (tmax[i] + L - 1) / L;
+      v[i] = (int)(s < 1 ? 1 : s > kMaxSplits ? kMaxSplits : s);
+    }
+    add(v);
+  }
+  std::sort(cands.begin(), cands.end(), [](const Cand& x, const Cand& y) { return x.lb < y.lb; });
+  std::vector<double> heap;
+  const Cand* best = &cands[0];
+  double best_us = -1.0;
+  for (const Cand& c : cands) {
+    if (best_us >= 0.0 && c.lb >= best_us) break;
+    double us = schedule_us(a, c.ns, n_heads, sms, heap);
+    for (int i = 0; i < a.n; ++i) us += merge_us((double)a.rows_per * n_heads, c.ns[i]);
+    if (best_us < 0.0 || us < best_us) {
+      best = &c;
+      best_us = us;
+    }
+  }
+  int mx = 1;
+  for (int i = 0; i < a.n; ++i) {
+    ns[i] = best->ns[i];
+    mx = ns[i] > mx ? ns[i] : mx;
+  }
+  return mx;
 }
 
 // q: map over [rows][H][128]; k, v: maps over the key rows ([rows][H][128]).
 int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                        const AttnDesc& a, int kv_row0, int n_heads, int n_splits, void* o,
+                        const AttnDesc& a, int kv_row0, int n_heads, const int* ns, void* o,
                         float* o_part, float* lse_part, const Guard& gd, cudaStream_t s) {
   const long long total_rows = (long long)a.n * a.rows_per;
   if (total_rows == 0) return SFM_OK;
   atc::Args args{};
   args.a = a;
   args.H = n_heads;
-  args.n_splits = n_splits;
   args.qtiles = (a.rows_per + atc::ROWS - 1) / atc::ROWS;
+  int max_splits = 1;
+  long long ctas = 0;
+  for (int i = 0; i < a.n; ++i) {
+    if (ns[i] < 1 || ns[i] > kMaxSplits) return SFM_EINVAL;
+    args.ns[i] = ns[i];
+    max_splits = ns[i] > max_splits ? ns[i] : max_splits;
+    ctas += (long long)ns[i] * n_heads * args.qtiles;
+  }
+  cta_order(a, ns, args.order);
   args.scale_log2 = (float)(1.4426950408889634 / sqrt((double)atc::D));
   args.total_rows = total_rows;
   args.kv_row0 = kv_row0;
@@ -629,17 +791,32 @@ int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
   args.err = gd.err;
   args.wait_ns = gd.wait_ns;
   args.fault = gd.fault;
-  dim3 grid(a.n * args.qtiles, n_heads, n_splits);
   cudaFuncSetAttribute(atc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, atc::SMEM);
   int rc;
   {
     ProfScope ps(SFM_PROF_ATTN, s);
-    atc::attn_tc_kernel<<<grid, atc::THREADS, atc::SMEM, s>>>(mq, mk, mv, args);
+    atc::attn_tc_kernel<<<(unsigned)ctas, atc::THREADS, atc::SMEM, s>>>(mq, mk, mv, args);
     rc = record_cuda(cudaGetLastError());
   }
-  if (rc || n_splits == 1) return rc;
+  if (rc || max_splits == 1) return rc;
+  // one merge per split count > 1 among the sessions (one-split sessions are done)
   ProfScope ps(SFM_PROF_ATTN_MERGE, s);
-  return launch_attention_merge(o_part, lse_part, o, total_rows, n_heads, n_splits, s);
+  for (int c = 2; c <= max_splits && !rc; ++c) {
+    MergeDesc md{};
+    md.rows_per = a.rows_per;
+    for (int i = 0; i < a.n; ++i)
+      if (ns[i] == c) md.sess[md.n++] = i;
+    if (md.n) rc = launch_attention_merge(o_part, lse_part, o, total_rows, n_heads, c, md, s);
+  }
+  return rc;
+}
+
+int launch_attention_tc(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const AttnDesc& a, int kv_row0, int n_heads, int n_splits, void* o,
+                        float* o_part, float* lse_part, const Guard& gd, cudaStream_t s) {
+  int ns[kMaxBatch];
+  for (int i = 0; i < kMaxBatch; ++i) ns[i] = n_splits;
+  return launch_attention_tc(mq, mk, mv, a, kv_row0, n_heads, ns, o, o_part, lse_part, gd, s);
 }
 
 }  // namespace sfm

@@ -93,3 +93,41 @@ def test_attention_workspace_grows_with_splits():
     big = L.lib.sfm_attention_workspace_bytes(924, 132924, 24, 128, L.SFM_DTYPE_BF16)
     assert big >= small
     assert big % 16 == 0
+
+
+def test_attention_batch_splits_per_session():
+    # host-only plan of the batched attention: one split count per session
+    ws = L.lib.sfm_attention_workspace_bytes(924, 58524, 24, 128, L.SFM_DTYPE_BF16)
+    single = ws // (924 * 24 * 129 * 4)
+    # one session: the standalone call's count (its workspace holds that many partials)
+    assert L.attention_batch_splits(924, [58524], 24) == [single]
+    # identical sessions share one count
+    same = L.attention_batch_splits(924, [58524] * 8, 24)
+    assert len(set(same)) == 1
+    # eight ragged caches of 24K-58K tokens (640x368 units): counts differ, and a longer
+    # session never gets fewer splits than a shorter one
+    keys = [c * 1200 + 924 for c in (38, 20, 25, 22, 20, 48, 35, 42)]
+    sp = L.attention_batch_splits(924, keys, 24)
+    assert len(set(sp)) > 1 and all(1 <= s <= 16 for s in sp)
+    for a in range(8):
+        for b in range(8):
+            if keys[a] < keys[b]:
+                assert sp[a] <= sp[b], (keys, sp)
+    # every split keeps at least two key tiles of 128
+    for k, s in zip(keys, sp):
+        assert s == 1 or (k + 127) // 128 // s >= 2
+    # a batch mixing one-split sessions (output written by the attention kernel) with
+    # merged ones: the small-width batched parity test relies on this plan
+    mix = L.attention_batch_splits(204, [1 * 100 + 204, 10 * 100 + 204, 60 * 100 + 204], 4)
+    assert mix[0] == 1 and mix[2] > 1, mix
+
+
+@pytest.mark.parametrize("n,rows,keys,heads,sms", [
+    (0, 924, [100], 24, 148), (17, 924, [100] * 17, 24, 148), (1, 0, [100], 24, 148),
+    (1, 924, [0], 24, 148), (1, 924, [100], 0, 148), (1, 924, [100], 24, 0)])
+def test_attention_batch_splits_rejects_bad_arguments(n, rows, keys, heads, sms):
+    k = (C.c_longlong * max(1, len(keys)))(*keys)
+    out = (C.c_int * 17)()
+    assert L.lib.sfm_attention_batch_splits(n, rows, k, heads, sms, out) == L.SFM_EINVAL
+    assert L.lib.sfm_attention_batch_splits(1, 924, None, 24, 148, out) == L.SFM_EINVAL
+    assert L.lib.sfm_attention_batch_splits(1, 924, k, 24, 148, None) == L.SFM_EINVAL

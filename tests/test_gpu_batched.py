@@ -87,3 +87,46 @@ def test_batched_argument_errors(cuda_device):
     zsame = (C.c_void_p * 2)(z[0].data_ptr(), z[0].data_ptr())
     assert L.lib.sfm_fm_solve_batched(p._h, 2, arr2, zsame, taus, 3, st) == L.SFM_EINVAL
     p.close()
+
+
+def test_batch_mixing_one_split_and_merged_sessions(cuda_device):
+    # caches of 1, 10 and 60 units: the batched attention gives the shortest session
+    # one key split (its output written by the attention kernel itself) and the others
+    # several, merged afterwards -- each session against its own solve and the oracle
+    from streaming_flow_matching_b200 import Performer
+    w = SMALL_BF16
+    caps = [1, 10, 60]
+    plan = L.attention_batch_splits(w.n_tokens, [c * w.unit_kv_tokens + w.n_tokens for c in caps],
+                                    w.n_heads, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert plan[0] == 1 and plan[2] > 1, plan
+    weights_cpu = S.make_weights(w)
+    pool = sum(c * w.unit_kv_tokens + w.n_tokens for c in caps)
+    p = Performer.from_workload(w, to_cuda(weights_cpu), pool_tokens=pool, max_sessions=3)
+    sessions, slices = [], []
+    for i, cap in enumerate(caps):
+        s = p.open_session(cap)
+        k, v = S.make_kv_slices(w, cap, seed=300 + i)
+        p.kvcache_append(s, k.cuda(), v.cuda())
+        sessions.append(s)
+        slices.append((k, v))
+    _, eps = S.make_latents(w, n_sessions=len(caps))
+    taus = S.uniform_taus(w.n_steps)
+    zs = [eps[i].cuda().clone() for i in range(len(caps))]
+    p.fm_solve_batched(sessions, zs, taus)
+    singles = []
+    for i, s in enumerate(sessions):
+        z = eps[i].cuda().clone()
+        p.fm_solve(s, z, taus)
+        singles.append(z)
+    torch.cuda.synchronize()
+    assert p.check_device_error() == 0
+    for i, s in enumerate(sessions):
+        assert rel_l2(zs[i].cpu().numpy(), singles[i].cpu().numpy()) <= 2e-3
+        info = p.session_info(s)
+        k, v = slices[i]
+        ref = O.denoise_solve(ocfg(w), eps[i], taus, weights_cpu, [k[l] for l in range(k.shape[0])],
+                              [v[l] for l in range(v.shape[0])], info["valid_tokens"], info["p0"])
+        e = rel_l2(zs[i].cpu().numpy(), ref)
+        print(f"session {i}: {caps[i]} units, {plan[i]} split(s): rel L2 {e:.3e}")
+        assert e <= BF16_TOL
+    p.close()

@@ -120,6 +120,10 @@ def test_attention_batch_splits_per_session():
     # merged ones: the small-width batched parity test relies on this plan
     mix = L.attention_batch_splits(204, [1 * 100 + 204, 10 * 100 + 204, 60 * 100 + 204], 4)
     assert mix[0] == 1 and mix[2] > 1, mix
+    # a guided pair at 640x368 (conditional: full cache; unconditional: the unit alone): the
+    # unconditional entry needs no merge and the conditional one keeps the single session's count
+    guided = L.attention_batch_splits(924, [58524, 924], 24)
+    assert guided == [single, 1], guided
 
 
 @pytest.mark.parametrize("n,rows,keys,heads,sms", [
